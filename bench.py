@@ -1,0 +1,374 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused Kronecker transform + INT4 path on B200.
+
+Workload: the hidden-size-8192 configuration -- T = 8192 tokens of
+n = 8192 (= 64 x 128) bf16, per-channel cinv, alpha = 0.85.  One step is one
+kq_transform_quant call over the T tokens (the whole path: scale, both
+contractions, absmax, quantise, pack).  Inputs rotate over buffer sets whose
+total exceeds 2x the L2 size, so each step reads x from HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 it runs under torch.distributed (one process per GPU, NCCL); every
+rank processes its own shard of T tokens (weak scaling, no data-path
+collective); the timed region is bracketed by barriers and the reported time
+is the max over ranks.  ``--impl reference`` times the fp64 CPU oracle on the
+host cores instead (rank 0 only).  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kronecker_factored_transforms_b200.workloads import (make_workload, workload_bytes,  # noqa: E402
+                                                          workload_flops)
+
+WORKLOAD = "hidden8192"
+METRIC = "tokens/s and % roofline (HBM/tensor) for fused Kronecker transform+INT4 at n=8192"
+UNIT = "tokens/s"
+PROFILES = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = ["kronecker_factored_transforms_b200/csrc/kq_tc05.cu",
+                  "kronecker_factored_transforms_b200/csrc/kq_tc05_ptx.cuh",
+                  "kronecker_factored_transforms_b200/csrc/kq_warp_mma.cu",
+                  "kronecker_factored_transforms_b200/csrc/kq_common.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def config_dict(w, extra=None):
+    d = {"workload": "%s: T=%d tokens/GPU, n=%d (n1=%d, n2=%d), cinv per channel, alpha=%g"
+         % (WORKLOAD, w.T, w.n, w.n1, w.n2, w.alpha),
+         "T": w.T, "n": w.n, "n1": w.n1, "n2": w.n2, "alpha": w.alpha, "cinv": w.cinv is not None}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        p = os.path.join(ROOT, rel)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    p = os.path.join(PROFILES, "traffic_%s.json" % WORKLOAD)
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("kernel") != kernel_name or d.get("source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and the reference arm).
+
+def time_oracle(w, seconds, max_tokens=None):
+    import oracle
+    oracle.build()
+    nth = oracle.default_threads()
+    probe = min(w.T, max(nth, 16))
+    t0 = time.perf_counter()
+    oracle.transform_quant(w.x[:probe], w.P1, w.P2, w.cinv, w.alpha, w.n1, w.n2, nthreads=nth,
+                           want_codes=False)
+    dt = time.perf_counter() - t0
+    per_tok = dt / probe
+    sample = int(min(w.T, max(probe, seconds / max(per_tok, 1e-9))))
+    if max_tokens:
+        sample = min(sample, max_tokens)
+    t0 = time.perf_counter()
+    oracle.transform_quant(w.x[:sample], w.P1, w.P2, w.cinv, w.alpha, w.n1, w.n2, nthreads=nth,
+                           want_codes=False)
+    el = time.perf_counter() - t0
+    return sample / el, nth, sample, el
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = make_workload(WORKLOAD)
+    import oracle
+    oracle.build()
+    nth = oracle.default_threads()
+    # size each step so that warm-up + timed steps stay within ~2 minutes
+    probe = min(w.T, max(nth, 16))
+    t0 = time.perf_counter()
+    oracle.transform_quant(w.x[:probe], w.P1, w.P2, w.cinv, w.alpha, w.n1, w.n2, nthreads=nth,
+                           want_codes=False)
+    per_tok = (time.perf_counter() - t0) / probe
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    sample = int(max(1, min(w.T, budget / max(per_tok, 1e-9))))
+    for _ in range(args.warmup):
+        oracle.transform_quant(w.x[:sample], w.P1, w.P2, w.cinv, w.alpha, w.n1, w.n2, nthreads=nth,
+                               want_codes=False)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.transform_quant(w.x[:sample], w.P1, w.P2, w.cinv, w.alpha, w.n1, w.n2, nthreads=nth,
+                               want_codes=False)
+    el = time.perf_counter() - t0
+    value = sample * args.steps / el
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(w, {"sample_tokens_per_step": sample}),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nth, "kind": "oracle",
+                             "sample": "first %d of %d tokens per step, fp64 C oracle, %d threads"
+                                       % (sample, w.T, nth)},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region (NVML, read-only).
+
+class ClockSampler:
+    REASONS = {"gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+               "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+               "display_clock_setting": 0x100}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def sample(self):
+        if not self.ok:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+        except Exception:
+            pass
+
+    def _loop(self):
+        while not self._stop.wait(0.02):
+            self.sample()
+
+    def __enter__(self):
+        self.sample()
+        self._t = threading.Thread(target=self._loop, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join()
+        self.sample()
+
+    def report(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        names = [k for k, v in self.REASONS.items() if self.reasons & v and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    from kronecker_factored_transforms_b200 import _lib
+
+    w = make_workload(WORKLOAD, shard=rank)
+    T, n1, n2, n = w.T, w.n1, w.n2, w.n
+    kernel = _lib.kq_kernel_name(n1, n2, w.cinv is not None)
+
+    # Rotating device buffer sets: total > 2x L2 so x comes from HBM every step.
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    set_bytes = T * n * 2 + T * n // 2 + T * 4
+    R = max(2, math.ceil(2 * l2 / set_bytes) + 1)
+    x0 = torch.from_numpy(w.x.view(np.int16)).to(dev)
+    xs = [x0] + [x0.clone() for _ in range(R - 1)]
+    qs = [torch.empty((T, n // 2), dtype=torch.uint8, device=dev) for _ in range(R)]
+    ss = [torch.empty((T,), dtype=torch.float32, device=dev) for _ in range(R)]
+    P1 = torch.from_numpy(w.P1.view(np.int16)).to(dev)
+    P2 = torch.from_numpy(w.P2.view(np.int16)).to(dev)
+    cinv = torch.from_numpy(w.cinv).to(dev) if w.cinv is not None else None
+
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+    fn = _lib.lib.kq_transform_quant
+    ptrs = [(xs[i].data_ptr(), qs[i].data_ptr(), ss[i].data_ptr()) for i in range(R)]
+    p1, p2, ci = P1.data_ptr(), P2.data_ptr(), cinv.data_ptr() if cinv is not None else None
+    alpha = w.alpha
+
+    def step(i):
+        xp, qp, sp = ptrs[i % R]
+        st = fn(xp, p1, p2, ci, alpha, qp, sp, T, n1, n2, sptr)
+        if st != 0:
+            raise RuntimeError("kq_transform_quant: %s" % _lib.kq_status_string(st))
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with sampler:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if _lib.kq_device_error(stream) != 0:
+        raise RuntimeError("a bounded wait timed out inside the kernel")
+
+    # End to end through the C ABI from pinned host buffers: H2D inputs,
+    # kernel, D2H codes + scales, every step.
+    hx = torch.from_numpy(w.x.view(np.int16)).pin_memory()
+    hp1 = torch.from_numpy(w.P1.view(np.int16)).pin_memory()
+    hp2 = torch.from_numpy(w.P2.view(np.int16)).pin_memory()
+    hci = torch.from_numpy(w.cinv).pin_memory() if w.cinv is not None else None
+    hq = torch.empty((T, n // 2), dtype=torch.uint8).pin_memory()
+    hs = torch.empty((T,), dtype=torch.float32).pin_memory()
+    dx, dq, dsc = xs[0], qs[0], ss[0]
+
+    def e2e_step():
+        dx.copy_(hx, non_blocking=True)
+        P1.copy_(hp1, non_blocking=True)
+        P2.copy_(hp2, non_blocking=True)
+        if hci is not None:
+            cinv.copy_(hci, non_blocking=True)
+        _lib.kq_transform_quant(dx, P1, P2, cinv, alpha, dq, dsc, T, n1, n2, stream=sptr)
+        hq.copy_(dq, non_blocking=True)
+        hs.copy_(dsc, non_blocking=True)
+
+    h2d = hx.numel() * 2 + hp1.numel() * 2 + hp2.numel() * 2 + (hci.numel() * 4 if hci is not None else 0)
+    d2h = hq.numel() + hs.numel() * 4
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    clocks = sampler.report()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    ms_step = ms / args.steps
+    value = world * T * args.steps / (ms / 1e3)
+    hbm_peak, tf_peak, peak_kind = measured_peaks()
+    bytes_launch = workload_bytes(T, n)
+    flops_launch = workload_flops(T, n1, n2)
+    achieved = bytes_launch / (ms_step / 1e3) / 1e9
+    t_hbm = bytes_launch / (hbm_peak * 1e9)
+    t_tc = flops_launch / (tf_peak * 1e12)
+    roof = {"bound": "hbm" if t_hbm >= t_tc else "tensor", "achieved": achieved, "peak": hbm_peak,
+            "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": recorded_traffic(kernel),
+            "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
+            else "fallback 6650 GB/s",
+            "kernel": kernel, "bytes_per_launch": bytes_launch, "flops_per_launch": flops_launch,
+            "tensor_frac_algorithmic": (flops_launch / (ms_step / 1e3) / 1e12) / tf_peak,
+            "roofline_time_us": 1e6 * max(t_hbm, t_tc), "measured_time_us": 1e3 * ms_step}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_dict(w, {"parallelism": "token-row shards, %d rank(s)" % world,
+                                      "l2": "inputs rotate over %d buffer sets (%.0f MB > 2x L2)"
+                                            % (R, R * set_bytes / 1e6),
+                                      "kernel": kernel}),
+            "roofline": roof,
+            "e2e": {"value": world * T * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps, "clocks": clocks}
+    if world == 1 and not args.no_cpu_baseline:
+        v, cores, sample, el = time_oracle(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": "first %d of %d tokens, fp64 C oracle, %.1f s"
+                                          % (sample, T, el)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

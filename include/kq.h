@@ -1,0 +1,129 @@
+/*
+ * kq.h -- C ABI of libkq: fused Kronecker-factored transform + per-token
+ * INT4 quantisation on an NVIDIA B200 (sm_100a).
+ *
+ * The operation (FlatQuant page, "Kronecker factorization" and "The fused
+ * kernel"; Kronecker Product page, "Definition" and the identity
+ * vec(V)(P1 (x) P2) = vec(P1^T V P2)):
+ *
+ *   for every token row x (length n = n1*n2, bf16):
+ *     x'  = x * cinv                  (per-channel scale 1/c; cinv NULL: c = 1)
+ *     X~  = x' read row-major as an n1 x n2 matrix, X~[a][b] = x'[a*n2 + b]
+ *     Y~  = P1^T X~ P2                (= x' (P1 (x) P2)),  y[i*n2 + j] = Y~[i][j]
+ *     s   = alpha * max_k |y_k| / 7   (one fp32 scale per token; clip after the
+ *                                      transform: FlatQuant page, "Per-channel
+ *                                      scaling and learnable clipping")
+ *     q_k = clamp(round_half_even(y_k / s), -8, 7)   (q = 0 when s = 0)
+ *     byte k of the token's output = (q_{2k} & 0xF) | ((q_{2k+1} & 0xF) << 4)
+ *
+ * Numerics: bf16 operands, fp32 accumulation on the tensor cores.  Every
+ * operand that is rounded to bf16 on the way (Z = X~' P2, and x' when cinv
+ * is given) is carried as a hi + lo pair of bf16 values, so the fp32 result
+ * is accurate to about 2^-16 of the token's absmax.
+ *
+ * Conventions shared by every entry point:
+ *   - All data pointers are DEVICE pointers into memory the caller owns.
+ *     The library allocates nothing and keeps no per-call state.
+ *   - bf16 arrays are passed as uint16_t bit patterns.  Matrices are dense
+ *     and row-major with no padding between rows.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  Inputs are read-only; outputs must not
+ *     overlap inputs (checked: KQ_ERR_ARG).
+ *   - T == 0 is a no-op that returns KQ_OK without touching any pointer.
+ *   - Arguments are checked before anything is launched; on error nothing
+ *     runs and the status says why.  Faults inside a kernel surface at the
+ *     caller's next synchronisation, as with any CUDA kernel.
+ *   - Supported factor sizes: n1 and n2 multiples of 16 in [16, 128].
+ */
+#ifndef KQ_H
+#define KQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kq_status {
+    KQ_OK = 0,
+    KQ_ERR_NULL = -1,        /* a required pointer is NULL (with T > 0)             */
+    KQ_ERR_SHAPE = -2,       /* T < 0, n1 <= 0, n2 <= 0, or T*n1*n2 overflows      */
+    KQ_ERR_UNSUPPORTED = -3, /* n1 or n2 not a multiple of 16 in [16, 128]         */
+    KQ_ERR_ALIGN = -4,       /* a pointer is not aligned as documented             */
+    KQ_ERR_ARG = -5,         /* alpha not finite in (0, 1], or outputs overlap inputs */
+    KQ_ERR_CUDA = -6,        /* a CUDA runtime call or a kernel launch failed      */
+    KQ_ERR_TIMEOUT = -7      /* a bounded wait inside a kernel gave up (see
+                                kq_device_error)                                    */
+} kq_status;
+
+/* Same type as cudaStream_t, declared here so the header needs no CUDA headers. */
+typedef struct CUstream_st *kq_stream_t;
+
+/*
+ * kq_transform_quant -- the fused hot path.
+ *   x         [T, n1*n2] bf16, 16-byte aligned.
+ *   P1        [n1, n1] bf16 (left factor; applied transposed), 16-byte aligned.
+ *   P2        [n2, n2] bf16 (right factor), 16-byte aligned.
+ *   cinv      [n1*n2] fp32 = 1/c, 16-byte aligned, or NULL for c = 1.
+ *   alpha     clip ratio, finite, 0 < alpha <= 1.
+ *   q_out     [T, n1*n2/2] uint8 packed INT4 codes, 16-byte aligned.
+ *   scale_out [T] fp32 per-token scale s, 4-byte aligned.
+ * Only q_out and scale_out are written; no intermediate touches global memory.
+ */
+kq_status kq_transform_quant(const uint16_t *x, const uint16_t *P1, const uint16_t *P2,
+                             const float *cinv, float alpha, uint8_t *q_out, float *scale_out,
+                             int64_t T, int n1, int n2, kq_stream_t stream);
+
+/*
+ * kq_transform -- check entry: the same transform, y written out in fp32
+ * instead of being quantised.  y_out [T, n1*n2] fp32, 16-byte aligned.
+ * Other arguments as for kq_transform_quant.
+ */
+kq_status kq_transform(const uint16_t *x, const uint16_t *P1, const uint16_t *P2,
+                       const float *cinv, float *y_out, int64_t T, int n1, int n2,
+                       kq_stream_t stream);
+
+/*
+ * kq_dequant_inverse -- check entry: undo the quantised transform.
+ * The inverse of P1 (x) P2 is P1^-1 (x) P2^-1 (FlatQuant page, "Kronecker
+ * factorization"; the page inverts P through its SVD, "Learning the affine
+ * transformation"), so with Y^ = q * s:
+ *     x^~ = P1^-T Y^ P2^-1,   x^ = x^~ * c.
+ *   q      [T, n1*n2/2] packed codes as written by kq_transform_quant, 16-byte aligned.
+ *   scale  [T] fp32.
+ *   P1inv  [n1, n1] fp32, P2inv [n2, n2] fp32: inverses computed by the caller
+ *          (e.g. in fp64 on the host, then rounded to fp32).
+ *   c      [n1*n2] fp32 channel scale (the reciprocal of cinv), or NULL for c = 1.
+ *   x_hat  [T, n1*n2] fp32 output, 16-byte aligned.
+ * Arithmetic is fp32 on CUDA cores; this entry is a checker, not a hot path.
+ */
+kq_status kq_dequant_inverse(const uint8_t *q, const float *scale, const float *P1inv,
+                             const float *P2inv, const float *c, float *x_hat, int64_t T,
+                             int n1, int n2, kq_stream_t stream);
+
+/*
+ * kq_device_error -- read and clear the device-side status word that the
+ * kernels set when a bounded wait gives up (they then skip their remaining
+ * work instead of hanging).  Synchronises `stream`.  *code receives 0 when
+ * no wait timed out since the last call, else a nonzero site code.
+ * Returns KQ_ERR_NULL for a NULL code, KQ_ERR_CUDA if the read fails.
+ */
+kq_status kq_device_error(kq_stream_t stream, int *code);
+
+/* Human-readable text for a kq_status value (static storage, never NULL). */
+const char *kq_status_string(int status);
+
+/*
+ * Name of the kernel kq_transform_quant launches for this shape (static
+ * storage), or "unsupported".  Host-only; touches no device state.
+ */
+const char *kq_kernel_name(int n1, int n2, int has_cinv);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int kq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KQ_H */

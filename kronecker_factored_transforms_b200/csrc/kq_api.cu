@@ -1,0 +1,190 @@
+// kq_api.cu -- the extern "C" boundary of libkq (declared in include/kq.h).
+//
+// Every entry point validates its arguments on the host before anything is
+// launched, then picks a kernel for the shape and launches it on the
+// caller's stream.  Nothing is allocated and no per-call state is kept.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/kq.h"
+#include "kq_internal.h"
+
+namespace {
+
+constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+struct Range {
+    uintptr_t lo, hi;  // [lo, hi)
+};
+Range range_of(const void *p, uint64_t bytes) {
+    uintptr_t b = reinterpret_cast<uintptr_t>(p);
+    return Range{b, b + static_cast<uintptr_t>(bytes)};
+}
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.hi > a.lo && b.hi > b.lo; }
+
+bool supported_factor(int k) { return k >= 16 && k <= 128 && k % 16 == 0; }
+
+// Shape checks shared by all entries: SHAPE, then UNSUPPORTED, then overflow.
+kq_status check_shape(int64_t T, int n1, int n2) {
+    if (T < 0 || n1 <= 0 || n2 <= 0) return KQ_ERR_SHAPE;
+    if (!supported_factor(n1) || !supported_factor(n2)) return KQ_ERR_UNSUPPORTED;
+    const int64_t n = int64_t(n1) * n2;
+    if (T > INT64_MAX / (n * 4)) return KQ_ERR_SHAPE;  // largest buffer is T*n*4 bytes
+    return KQ_OK;
+}
+
+kq_status check_alpha(float alpha) {
+    if (!std::isfinite(alpha) || !(alpha > 0.0f) || alpha > 1.0f) return KQ_ERR_ARG;
+    return KQ_OK;
+}
+
+struct DeviceInfo {
+    int device = -1;
+    int num_sms = 0;
+};
+
+// SM count per device, queried once per device.
+kq_status device_info(DeviceInfo &info) {
+    static std::mutex mu;
+    static int sms_cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64) return KQ_ERR_CUDA;
+    if (sms_cache[dev] == 0) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return KQ_ERR_CUDA;
+        sms_cache[dev] = sms;
+    }
+    info.device = dev;
+    info.num_sms = sms_cache[dev];
+    return KQ_OK;
+}
+
+kq_status run_transform(const uint16_t *x, const uint16_t *P1, const uint16_t *P2, const float *cinv,
+                        float alpha, uint8_t *q_out, float *scale_out, float *y_out, int64_t T,
+                        int n1, int n2, kq_stream_t stream) {
+    DeviceInfo info;
+    kq_status st = device_info(info);
+    if (st != KQ_OK) return st;
+    kq::LaunchArgs a;
+    a.x = x;
+    a.P1 = P1;
+    a.P2 = P2;
+    a.cinv = cinv;
+    a.alpha = alpha;
+    a.q_out = q_out;
+    a.scale_out = scale_out;
+    a.y_out = y_out;
+    a.T = T;
+    a.n1 = n1;
+    a.n2 = n2;
+    a.num_sms = info.num_sms;
+    a.device = info.device;
+    a.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err = (y_out == nullptr && kq::tc05_supports(n1, n2, cinv != nullptr))
+                          ? kq::launch_tc05(a)
+                          : kq::launch_warp_mma(a);
+    return err == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+kq_status kq_transform_quant(const uint16_t *x, const uint16_t *P1, const uint16_t *P2,
+                             const float *cinv, float alpha, uint8_t *q_out, float *scale_out,
+                             int64_t T, int n1, int n2, kq_stream_t stream) {
+    kq_status st = check_shape(T, n1, n2);
+    if (st != KQ_OK) return st;
+    if ((st = check_alpha(alpha)) != KQ_OK) return st;
+    if (T == 0) return KQ_OK;
+    if (!x || !P1 || !P2 || !q_out || !scale_out) return KQ_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(P1, 16) || !aligned(P2, 16) || !aligned(q_out, 16) ||
+        !aligned(scale_out, 4) || (cinv && !aligned(cinv, 16)))
+        return KQ_ERR_ALIGN;
+    const uint64_t n = uint64_t(n1) * n2;
+    const Range in[4] = {range_of(x, uint64_t(T) * n * 2), range_of(P1, uint64_t(n1) * n1 * 2),
+                         range_of(P2, uint64_t(n2) * n2 * 2), range_of(cinv, cinv ? n * 4 : 0)};
+    const Range rq = range_of(q_out, uint64_t(T) * n / 2), rs = range_of(scale_out, uint64_t(T) * 4);
+    for (const Range &r : in)
+        if (overlap(r, rq) || overlap(r, rs)) return KQ_ERR_ARG;
+    if (overlap(rq, rs)) return KQ_ERR_ARG;
+    return run_transform(x, P1, P2, cinv, alpha, q_out, scale_out, nullptr, T, n1, n2, stream);
+}
+
+kq_status kq_transform(const uint16_t *x, const uint16_t *P1, const uint16_t *P2, const float *cinv,
+                       float *y_out, int64_t T, int n1, int n2, kq_stream_t stream) {
+    kq_status st = check_shape(T, n1, n2);
+    if (st != KQ_OK) return st;
+    if (T == 0) return KQ_OK;
+    if (!x || !P1 || !P2 || !y_out) return KQ_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(P1, 16) || !aligned(P2, 16) || !aligned(y_out, 16) ||
+        (cinv && !aligned(cinv, 16)))
+        return KQ_ERR_ALIGN;
+    const uint64_t n = uint64_t(n1) * n2;
+    const Range in[4] = {range_of(x, uint64_t(T) * n * 2), range_of(P1, uint64_t(n1) * n1 * 2),
+                         range_of(P2, uint64_t(n2) * n2 * 2), range_of(cinv, cinv ? n * 4 : 0)};
+    const Range ry = range_of(y_out, uint64_t(T) * n * 4);
+    for (const Range &r : in)
+        if (overlap(r, ry)) return KQ_ERR_ARG;
+    return run_transform(x, P1, P2, cinv, 1.0f, nullptr, nullptr, y_out, T, n1, n2, stream);
+}
+
+kq_status kq_dequant_inverse(const uint8_t *q, const float *scale, const float *P1inv,
+                             const float *P2inv, const float *c, float *x_hat, int64_t T, int n1,
+                             int n2, kq_stream_t stream) {
+    kq_status st = check_shape(T, n1, n2);
+    if (st != KQ_OK) return st;
+    if (T == 0) return KQ_OK;
+    if (!q || !scale || !P1inv || !P2inv || !x_hat) return KQ_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(scale, 4) || !aligned(P1inv, 4) || !aligned(P2inv, 4) ||
+        !aligned(x_hat, 16) || (c && !aligned(c, 4)))
+        return KQ_ERR_ALIGN;
+    const uint64_t n = uint64_t(n1) * n2;
+    const Range in[5] = {range_of(q, uint64_t(T) * n / 2), range_of(scale, uint64_t(T) * 4),
+                         range_of(P1inv, uint64_t(n1) * n1 * 4), range_of(P2inv, uint64_t(n2) * n2 * 4),
+                         range_of(c, c ? n * 4 : 0)};
+    const Range rx = range_of(x_hat, uint64_t(T) * n * 4);
+    for (const Range &r : in)
+        if (overlap(r, rx)) return KQ_ERR_ARG;
+    cudaError_t err = kq::launch_dequant_inverse(q, scale, P1inv, P2inv, c, x_hat, T, n1, n2,
+                                                 reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;
+}
+
+kq_status kq_device_error(kq_stream_t stream, int *code) {
+    if (!code) return KQ_ERR_NULL;
+    unsigned int v = 0;
+    if (kq::read_and_clear_device_error(reinterpret_cast<cudaStream_t>(stream), &v) != cudaSuccess)
+        return KQ_ERR_CUDA;
+    *code = static_cast<int>(v);
+    return KQ_OK;
+}
+
+const char *kq_status_string(int status) {
+    switch (status) {
+    case KQ_OK: return "ok";
+    case KQ_ERR_NULL: return "a required pointer is NULL";
+    case KQ_ERR_SHAPE: return "bad shape (T < 0, n1 <= 0, n2 <= 0 or size overflow)";
+    case KQ_ERR_UNSUPPORTED: return "unsupported factor size (n1, n2 must be multiples of 16 in [16, 128])";
+    case KQ_ERR_ALIGN: return "misaligned pointer";
+    case KQ_ERR_ARG: return "bad argument (alpha outside (0, 1] or outputs overlap inputs)";
+    case KQ_ERR_CUDA: return "CUDA runtime error";
+    case KQ_ERR_TIMEOUT: return "a bounded wait inside a kernel timed out";
+    default: return "unknown status";
+    }
+}
+
+const char *kq_kernel_name(int n1, int n2, int has_cinv) {
+    if (!supported_factor(n1) || !supported_factor(n2)) return "unsupported";
+    return kq::tc05_supports(n1, n2, has_cinv != 0) ? "kq_tc05_fused_kernel" : "kq_warp_mma_kernel";
+}
+
+int kq_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,40 @@
+// kq_internal.h -- launch plumbing shared between the C ABI and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kq {
+
+struct LaunchArgs {
+    const uint16_t *x;
+    const uint16_t *P1;
+    const uint16_t *P2;
+    const float *cinv;   // nullptr: c = 1
+    float alpha;
+    uint8_t *q_out;      // quantise mode
+    float *scale_out;
+    float *y_out;        // transform-only mode when non-null
+    int64_t T;
+    int n1, n2;
+    int num_sms;
+    int device;
+    cudaStream_t stream;
+};
+
+// General warp-level MMA kernel: every supported shape.
+cudaError_t launch_warp_mma(const LaunchArgs &a);
+
+// Persistent tcgen05/TMEM kernel for the shapes it covers.
+bool tc05_supports(int n1, int n2, bool scaled);
+cudaError_t launch_tc05(const LaunchArgs &a);
+
+// Read and clear the device status word set by bounded waits that gave up.
+cudaError_t read_and_clear_device_error(cudaStream_t stream, unsigned int *code);
+
+// Check entry: q * s -> P1inv^T Y P2inv -> * c, fp32 on CUDA cores.
+cudaError_t launch_dequant_inverse(const uint8_t *q, const float *scale, const float *P1inv,
+                                   const float *P2inv, const float *c, float *x_hat, int64_t T,
+                                   int n1, int n2, cudaStream_t stream);
+
+}  // namespace kq

@@ -13,7 +13,9 @@ per-channel scaling c) stand in for real LLM activations, which are not used.
 
 Conventions (one reading, fixed here and restated in the design doc):
   * numpy ``default_rng(seed)`` (PCG64); draw order P1, P2, outlier channel
-    set, x (in chunks of ``CHUNK_ROWS`` rows), then c.
+    set, c, then x (in chunks of ``CHUNK_ROWS`` rows).
+  * shard r > 0 of a multi-GPU run draws its rows of x from
+    ``default_rng([seed, r])``; factors, outlier channels and c are shared.
   * bf16 = round-to-nearest-even of the float32 value.
   * orthogonal factor: Q of QR(Gaussian) with columns multiplied by
     sign(diag R), cast to bf16 (so it is only nearly orthogonal).
@@ -125,13 +127,16 @@ CONFIGS = {
 SWEEP_T = (1, 16, 128, 1024, 16384, 65536)
 
 
-def make_workload(name: str, T: Optional[int] = None, rows: Optional[int] = None) -> Workload:
+def make_workload(name: str, T: Optional[int] = None, rows: Optional[int] = None,
+                  shard: int = 0) -> Workload:
     """Build config ``name`` (see ``CONFIGS``) with its seed.
 
     ``T`` overrides the token count (the same seed gives the same factors and
     the same leading rows of x for every T).  ``rows`` generates only the
     first ``rows`` tokens of a T-token workload (identical to the leading
     rows of the full one): a cheap way to sample a large configuration.
+    ``shard`` selects an independent block of rows with the same factors,
+    outlier channels and c (one block per rank in a multi-GPU run).
     """
     cfg = CONFIGS[name]
     T = int(cfg["T"] if T is None else T)
@@ -152,39 +157,34 @@ def make_workload(name: str, T: Optional[int] = None, rows: Optional[int] = None
     else:
         chan, factor = _outlier_channels(rng, n, float(out[1])), float(out[2])
 
+    cinv = None
+    if cfg["scaled"]:
+        c = np.exp(rng.uniform(math.log(0.5), math.log(2.0), size=n))
+        cinv = (1.0 / c).astype(np.float32)
+
+    xrng = rng if shard == 0 else np.random.default_rng([cfg["seed"], int(shard)])
     x_bits = np.empty((rows_out, n), dtype=np.uint16)
     done = 0
     while done < rows_out:
         r = min(CHUNK_ROWS, T - done)
         kind = cfg["x_kind"]
         if kind == "normal":
-            blk = rng.standard_normal((r, n))
+            blk = xrng.standard_normal((r, n))
         elif kind == "student_t":
-            blk = 0.5 * rng.standard_t(3, size=(r, n))
+            blk = 0.5 * xrng.standard_t(3, size=(r, n))
         elif kind == "relu_gated":
-            g = rng.standard_normal((r, n)) * math.sqrt(2.0)
-            mask = rng.random((r, n)) < 0.5
+            g = xrng.standard_normal((r, n)) * math.sqrt(2.0)
+            mask = xrng.random((r, n)) < 0.5
             blk = np.where(mask, g, 0.0)
         else:  # pragma: no cover - recipe table is closed
             raise ValueError(kind)
         if chan.size:
             blk[:, chan] *= factor
-        if cfg["pivot"] is not None and done == 0:
+        if cfg["pivot"] is not None and done == 0 and shard == 0:
             blk[0, :] *= cfg["pivot"]
         take = min(r, rows_out - done)
         x_bits[done:done + take] = f32_to_bf16_bits(blk[:take].astype(np.float32))
         done += r
-
-    cinv = None
-    if cfg["scaled"]:
-        # c is drawn after x: consume the rows of x that were not generated
-        # so that c does not depend on ``rows``.
-        while done < T:
-            r = min(CHUNK_ROWS, T - done)
-            rng.standard_t(3, size=(r, n))
-            done += r
-        c = np.exp(rng.uniform(math.log(0.5), math.log(2.0), size=n))
-        cinv = (1.0 / c).astype(np.float32)
 
     return Workload(name=name, T=T, n1=n1, n2=n2, x=x_bits,
                     P1=f32_to_bf16_bits(P1.astype(np.float32)),

@@ -1,0 +1,122 @@
+"""The C-ABI library: it loads, exports what include/kq.h declares, and rejects
+bad arguments on the host before anything is launched (no GPU needed: every
+call below fails validation, so no CUDA call is made)."""
+import math
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kq.h")
+
+
+@pytest.fixture(scope="module")
+def kq():
+    from kronecker_factored_transforms_b200 import build
+    build.build()
+    from kronecker_factored_transforms_b200 import _lib
+    return _lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kq_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for must in ("kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_status_string",
+                 "kq_kernel_name", "kq_device_error", "kq_version"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(kq):
+    out = subprocess.run(["nm", "-D", "--defined-only", kq.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT\s+(kq_[a-z_0-9]+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        getattr(kq.lib, name)
+
+
+def test_version_and_strings(kq):
+    assert kq.kq_version() >= 10000
+    for st in range(-7, 1):
+        assert kq.kq_status_string(st) not in ("", "unknown status")
+    assert kq.kq_status_string(42) == "unknown status"
+
+
+def test_kernel_name_for_shapes(kq):
+    assert kq.kq_kernel_name(16, 16, False) != "unsupported"
+    assert kq.kq_kernel_name(64, 128, True) != "unsupported"
+    assert kq.kq_kernel_name(112, 128, False) != "unsupported"
+    assert kq.kq_kernel_name(24, 16, False) == "unsupported"
+    assert kq.kq_kernel_name(16, 144, False) == "unsupported"
+
+
+# Fake, never-dereferenced device addresses (validation rejects every call below).
+X, P1, P2, CI, Q, S, Y = 0x10000000, 0x20000000, 0x20010000, 0x20020000, 0x30000000, 0x40000000, 0x50000000
+
+
+def tq(kq, **kw):
+    a = dict(x=X, P1=P1, P2=P2, cinv=CI, alpha=0.9, q=Q, s=S, T=8, n1=64, n2=128)
+    a.update(kw)
+    return kq.lib.kq_transform_quant(a["x"], a["P1"], a["P2"], a["cinv"], a["alpha"], a["q"], a["s"],
+                                     a["T"], a["n1"], a["n2"], None)
+
+
+def test_transform_quant_validation(kq):
+    assert tq(kq, T=-1) == kq.KQ_ERR_SHAPE
+    assert tq(kq, n1=0) == kq.KQ_ERR_SHAPE
+    assert tq(kq, n2=-16) == kq.KQ_ERR_SHAPE
+    for bad in (8, 24, 144, 256):
+        assert tq(kq, n1=bad) == kq.KQ_ERR_UNSUPPORTED
+        assert tq(kq, n2=bad) == kq.KQ_ERR_UNSUPPORTED
+    for bad in (0.0, -0.5, 1.0000001, 2.0, math.nan, math.inf):
+        assert tq(kq, alpha=bad) == kq.KQ_ERR_ARG
+    assert tq(kq, T=2 ** 62) == kq.KQ_ERR_SHAPE
+    # T == 0 is a no-op even with NULL pointers.
+    assert tq(kq, T=0, x=None, P1=None, P2=None, cinv=None, q=None, s=None) == kq.KQ_OK
+    for name in ("x", "P1", "P2", "q", "s"):
+        assert tq(kq, **{name: None}) == kq.KQ_ERR_NULL
+    for name in ("x", "P1", "P2", "q", "cinv"):
+        assert tq(kq, **{name: {"x": X, "P1": P1, "P2": P2, "q": Q, "cinv": CI}[name] + 8}) == kq.KQ_ERR_ALIGN
+    assert tq(kq, s=S + 2) == kq.KQ_ERR_ALIGN
+    # Outputs overlapping inputs (or each other).
+    assert tq(kq, q=X + 64) == kq.KQ_ERR_ARG
+    assert tq(kq, s=P1 + 16) == kq.KQ_ERR_ARG
+    assert tq(kq, s=Q + 16) == kq.KQ_ERR_ARG
+    assert tq(kq, q=CI) == kq.KQ_ERR_ARG
+
+
+def test_transform_validation(kq):
+    f = kq.lib.kq_transform
+    assert f(X, P1, P2, None, Y, -3, 64, 64, None) == kq.KQ_ERR_SHAPE
+    assert f(X, P1, P2, None, Y, 3, 40, 64, None) == kq.KQ_ERR_UNSUPPORTED
+    assert f(X, P1, P2, None, None, 3, 64, 64, None) == kq.KQ_ERR_NULL
+    assert f(X, P1, P2, None, Y + 4, 3, 64, 64, None) == kq.KQ_ERR_ALIGN
+    assert f(X, P1, P2, None, X + 16, 3, 64, 64, None) == kq.KQ_ERR_ARG
+    assert f(None, None, None, None, None, 0, 64, 64, None) == kq.KQ_OK
+
+
+def test_dequant_inverse_validation(kq):
+    f = kq.lib.kq_dequant_inverse
+    assert f(Q, S, P1, P2, None, Y, -1, 16, 16, None) == kq.KQ_ERR_SHAPE
+    assert f(Q, S, P1, P2, None, Y, 4, 16, 20, None) == kq.KQ_ERR_UNSUPPORTED
+    assert f(Q, None, P1, P2, None, Y, 4, 16, 16, None) == kq.KQ_ERR_NULL
+    assert f(Q + 1, S, P1, P2, None, Y, 4, 16, 16, None) == kq.KQ_ERR_ALIGN
+    assert f(Q, S, P1, P2, None, Q + 32, 4, 16, 16, None) == kq.KQ_ERR_ARG
+    assert f(None, None, None, None, None, None, 0, 16, 16, None) == kq.KQ_OK
+
+
+def test_device_error_rejects_null(kq):
+    assert kq.lib.kq_device_error(None, None) == kq.KQ_ERR_NULL
+
+
+def test_binding_raises_on_bad_status(kq):
+    with pytest.raises(kq.KQError) as e:
+        kq.kq_transform_quant(X, P1, P2, None, 0.9, Q, S, 4, 24, 16, stream=0)
+    assert e.value.status == kq.KQ_ERR_UNSUPPORTED
