@@ -110,6 +110,18 @@ kq_status kq_dequant_inverse(const uint8_t *q, const float *scale, const float *
  */
 kq_status kq_device_error(kq_stream_t stream, int *code);
 
+/*
+ * kq_selftest_bounded_wait -- diagnostic for the failure path of the bounded
+ * waits.  Launches one tiny kernel on `stream` whose thread waits on a
+ * shared-memory barrier that nothing ever signals; after `limit_us`
+ * microseconds (1 .. 10,000,000) the wait gives up, records site code 256 in
+ * the device status word and the kernel returns normally.  Nothing faults and
+ * the context stays usable; kq_device_error then reports 256.
+ * Returns KQ_ERR_ARG for a limit outside the range, KQ_ERR_CUDA if the launch
+ * fails.
+ */
+kq_status kq_selftest_bounded_wait(int64_t limit_us, kq_stream_t stream);
+
 /* Human-readable text for a kq_status value (static storage, never NULL). */
 const char *kq_status_string(int status);
 

@@ -6,7 +6,7 @@ ctypes binding (``_lib``) and the seeded synthetic input generator
 (``workloads``).  Importing the binding requires the built library.
 """
 __all__ = ["kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_device_error",
-           "kq_status_string", "kq_kernel_name", "kq_version", "KQError"]
+           "kq_selftest_bounded_wait", "kq_status_string", "kq_kernel_name", "kq_version", "KQError"]
 
 
 def __getattr__(name):

@@ -40,7 +40,9 @@ def _load() -> ctypes.CDLL:
     lib.kq_transform.argtypes = [P, P, P, P, P, I64, I32, I32, P]
     lib.kq_dequant_inverse.argtypes = [P, P, P, P, P, P, I64, I32, I32, P]
     lib.kq_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
-    for f in (lib.kq_transform_quant, lib.kq_transform, lib.kq_dequant_inverse, lib.kq_device_error):
+    lib.kq_selftest_bounded_wait.argtypes = [I64, P]
+    for f in (lib.kq_transform_quant, lib.kq_transform, lib.kq_dequant_inverse, lib.kq_device_error,
+              lib.kq_selftest_bounded_wait):
         f.restype = ctypes.c_int
     lib.kq_status_string.argtypes = [I32]
     lib.kq_status_string.restype = ctypes.c_char_p
@@ -54,7 +56,7 @@ def _load() -> ctypes.CDLL:
 lib = _load()
 
 EXPORTED = ("kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_device_error",
-            "kq_status_string", "kq_kernel_name", "kq_version")
+            "kq_selftest_bounded_wait", "kq_status_string", "kq_kernel_name", "kq_version")
 
 
 def _ptr(t) -> Optional[int]:
@@ -103,6 +105,10 @@ def kq_device_error(stream=None) -> int:
     code = ctypes.c_int(0)
     _check("kq_device_error", lib.kq_device_error(_stream(stream), ctypes.byref(code)))
     return code.value
+
+
+def kq_selftest_bounded_wait(limit_us: int, stream=None) -> None:
+    _check("kq_selftest_bounded_wait", lib.kq_selftest_bounded_wait(int(limit_us), _stream(stream)))
 
 
 def kq_status_string(status: int) -> str:

@@ -166,6 +166,13 @@ kq_status kq_device_error(kq_stream_t stream, int *code) {
     return KQ_OK;
 }
 
+kq_status kq_selftest_bounded_wait(int64_t limit_us, kq_stream_t stream) {
+    if (limit_us < 1 || limit_us > 10000000) return KQ_ERR_ARG;
+    cudaError_t err = kq::launch_selftest_wait(uint64_t(limit_us) * 1000u,
+                                               reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;
+}
+
 const char *kq_status_string(int status) {
     switch (status) {
     case KQ_OK: return "ok";

@@ -29,6 +29,9 @@ cudaError_t launch_warp_mma(const LaunchArgs &a);
 bool tc05_supports(int n1, int n2, bool scaled);
 cudaError_t launch_tc05(const LaunchArgs &a);
 
+// Diagnostic: a kernel whose bounded wait on a never-signalled barrier gives up.
+cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
+
 // Read and clear the device status word set by bounded waits that gave up.
 cudaError_t read_and_clear_device_error(cudaStream_t stream, unsigned int *code);
 

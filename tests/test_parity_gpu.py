@@ -215,3 +215,25 @@ def test_dequant_inverse_matches_oracle_and_round_trips(kq):
     colsum = (np.abs(I1).sum(0)[:, None] * np.abs(I2).sum(0)[None, :]).ravel()
     bound = 0.5 * s.astype(np.float64)[:, None] * colsum[None, :] * c[None, :] * 1.001
     assert np.all(np.abs(got - x) <= bound + 1e-4 * np.abs(x).max())
+
+
+# ---------------------------------------------------------------------------
+# Kernel selection and the bounded-wait failure path.
+
+def test_fast_kernel_is_selected_for_the_configs(kq):
+    for n1, n2, scaled in [(64, 64, False), (64, 128, True), (112, 128, False)]:
+        assert kq.kq_kernel_name(n1, n2, scaled) == "kq_tc05_fused_kernel"
+    assert kq.kq_kernel_name(16, 16, False) == "kq_warp_mma_kernel"
+
+
+def test_bounded_wait_times_out_without_fault(kq):
+    """A wait on a barrier nobody signals gives up after the limit, reports its
+    site code through the status word, and leaves the context usable."""
+    assert kq.kq_device_error() == 0
+    kq.kq_selftest_bounded_wait(20000)  # 20 ms
+    assert kq.kq_device_error() == 256
+    assert kq.kq_device_error() == 0    # read clears it
+    w = make_workload("hidden8192", rows=8)
+    q, s = run_quant(kq, w.x, w.P1, w.P2, w.cinv, w.alpha, 8, 64, 128)
+    assert_quant_parity(w.x, w.P1, w.P2, w.cinv, w.alpha, 64, 128, q, s)
+    assert kq.kq_device_error() == 0
