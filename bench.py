@@ -55,6 +55,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling runs)")
     return ap.parse_args()
 
 
@@ -311,18 +312,20 @@ def main():
 
     h2d = hx.numel() * 2 + hp1.numel() * 2 + hp2.numel() * 2 + (hci.numel() * 4 if hci is not None else 0)
     d2h = hq.numel() + hs.numel() * 4
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = float("nan")
+    if not args.no_e2e:
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1)
     if world > 1:
         t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -358,7 +361,8 @@ def main():
                                             % (R, R * set_bytes / 1e6),
                                       "kernel": kernel}),
             "roofline": roof,
-            "e2e": {"value": world * T * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+            "e2e": None if args.no_e2e else
+                   {"value": world * T * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps, "clocks": clocks}
     if world == 1 and not args.no_cpu_baseline:
