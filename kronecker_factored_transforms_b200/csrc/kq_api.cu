@@ -86,7 +86,9 @@ kq_status run_transform(const uint16_t *x, const uint16_t *P1, const uint16_t *P
     a.num_sms = info.num_sms;
     a.device = info.device;
     a.stream = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t err = (y_out == nullptr && kq::tc05_supports(n1, n2, cinv != nullptr))
+    // The tcgen05 kernel rounds with a 1.5 * 2^23 shift, exact while |y / s| = 7 / alpha < 2^22.
+    const bool fast = y_out == nullptr && alpha >= 0x1p-19f && kq::tc05_supports(n1, n2, cinv != nullptr);
+    cudaError_t err = fast
                           ? kq::launch_tc05(a)
                           : kq::launch_warp_mma(a);
     return err == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;

@@ -25,7 +25,7 @@ struct LaunchArgs {
 // General warp-level MMA kernel: every supported shape.
 cudaError_t launch_warp_mma(const LaunchArgs &a);
 
-// Persistent tcgen05/TMEM kernel for the shapes it covers.
+// Persistent tcgen05/TMEM kernel for the shapes it covers (alpha >= 2^-19).
 bool tc05_supports(int n1, int n2, bool scaled);
 cudaError_t launch_tc05(const LaunchArgs &a);
 

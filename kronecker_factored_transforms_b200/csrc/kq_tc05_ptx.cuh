@@ -138,6 +138,27 @@ __device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t (&r)
                  : "memory");
 }
 
+// ---- packed fp32 pairs (two lanes of arithmetic per instruction) -------------
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f32x2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// ---- integer packing ----------------------------------------------------------
+// d = (c << 8) | (sat4(a) << 4) | sat4(b): two signed 4-bit codes, saturated to
+// [-8, 7], b in the low nibble; the low bits of c move up by one byte.
+__device__ __forceinline__ uint32_t pack_s4x2(int a, int b, uint32_t c) {
+    uint32_t d;
+    asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
 // ---- tcgen05.mma (kind::f16, bf16 x bf16 -> fp32, one CTA) -------------------
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
