@@ -128,14 +128,14 @@ struct Cfg {
     static constexpr int OFF_B2 = 0;
     static constexpr int OFF_A1 = align_up(OFF_B2 + NCH2 * N1 * 128, 1024);
     static constexpr int OFF_RAW = OFF_A1 + (A1_TMEM ? 0 : 32768);
-    static constexpr int FIXED = OFF_RAW + (SCALED ? SC * 2 * XTILE : 0) + STG + 2048;
+    static constexpr int FIXED = OFF_RAW + (SCALED ? SC * 2 * XTILE : 0) + 2 * STG + 2048;
     static constexpr int SX = imax(2, imin(8, (222 * 1024 - FIXED) / XTILE));  // raw x stages
     static constexpr int OFF_CONV = OFF_RAW + SX * XTILE;
     static constexpr int OFF_STG = OFF_CONV + (SCALED ? SC * 2 * XTILE : 0);
     static constexpr int NBAR = 2 * SX + 2 * SC + 3 * NB1 + 2 * NB2 + 1;
-    static constexpr int OFF_BAR = align_up(OFF_STG + STG, 16);
-    static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem base, abort flag, 4 maxima
-    static constexpr int SMEM = OFF_MISC + 32 + 1024;    // + slack for 1024-byte alignment
+    static constexpr int OFF_BAR = align_up(OFF_STG + 2 * STG, 16);  // two staging buffers
+    static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem base, abort flag, 2 x 4 maxima
+    static constexpr int SMEM = OFF_MISC + 48 + 1024;    // + slack for 1024-byte alignment
     // barrier indices
     static constexpr int FULL = 0, EMPTY = SX, CFULL = 2 * SX, CEMPTY = 2 * SX + SC;
     static constexpr int D1FULL = 2 * SX + 2 * SC, A2FULL = D1FULL + NB1, D1EMPTY = A2FULL + NB1;
@@ -165,15 +165,17 @@ __device__ __forceinline__ uint16_t a1_value(const uint16_t *__restrict__ P2, in
 }
 
 // v = hi + lo with hi = v truncated to bf16 (its top 16 bits) and lo = v - hi
-// (exact in fp32), then rounded to bf16: about 16 significant bits in all.
-// Takes two fp32 values as one 64-bit pair; returns the two hi values packed
-// (first in the low half) and the two lo ones.
+// (exact in fp32), then lo rounded to bf16 to nearest (ties away from zero,
+// by adding half an ulp to the magnitude bits): about 16 significant bits in
+// all, using only integer and fp32 pipes.  Takes two fp32 values as one
+// 64-bit pair; returns the two hi values packed (first in the low half) and
+// the two lo ones.
 __device__ __forceinline__ void split2(uint64_t v, uint32_t &hi, uint32_t &lo) {
     const uint32_t v0 = uint32_t(v), v1 = uint32_t(v >> 32);
     const uint64_t t = uint64_t(v0 & 0xFFFF0000u) | (uint64_t(v1 & 0xFFFF0000u) << 32);
     const uint64_t l = f32x2_sub(v, t);
     hi = __byte_perm(v0, v1, 0x7632);
-    lo = pack_bf16x2(__uint_as_float(uint32_t(l)), __uint_as_float(uint32_t(l >> 32)));
+    lo = __byte_perm(uint32_t(l) + 0x8000u, uint32_t(l >> 32) + 0x8000u, 0x7632);
 }
 
 // round_half_even(y * inv) as an int, valid for |y * inv| < 2^22 (alpha >= 2^-19):
@@ -181,6 +183,18 @@ __device__ __forceinline__ void split2(uint64_t v, uint32_t &hi, uint32_t &lo) {
 __device__ __forceinline__ int round_code(uint32_t ybits, float inv) {
     return __float_as_int(fmaf(__uint_as_float(ybits), inv, 12582912.0f)) - 0x4B400000;
 }
+
+// Position in a ring of n barrier-guarded slots: slot index and the parity of
+// the slot's current phase; advancing past the last slot flips the parity.
+struct Ring {
+    uint32_t idx = 0, phase = 0;
+    __device__ __forceinline__ void next(uint32_t n) {
+        if (++idx == n) {
+            idx = 0;
+            phase ^= 1u;
+        }
+    }
+};
 
 template <int N1, int N2, bool SCALED>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -207,16 +221,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < C::SX; ++s) {
             mbar_init(bar(C::FULL + s), 1);
-            mbar_init(bar(C::EMPTY + s), SCALED ? 128 : 1);
+            mbar_init(bar(C::EMPTY + s), 128);
         }
         for (int c = 0; c < C::SC; ++c) {
             mbar_init(bar(C::CFULL + c), 128);
-            mbar_init(bar(C::CEMPTY + c), 1);
+            mbar_init(bar(C::CEMPTY + c), 128);
         }
         for (int b = 0; b < C::NB1; ++b) {
             mbar_init(bar(C::D1FULL + b), 1);
             mbar_init(bar(C::A2FULL + b), 128);
-            mbar_init(bar(C::D1EMPTY + b), 1);
+            mbar_init(bar(C::D1EMPTY + b), 128);
         }
         for (int b = 0; b < C::NB2; ++b) {
             mbar_init(bar(C::D2FULL + b), 1);
@@ -270,18 +284,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
 
+    // Release of x tiles: stage 1 of a batch finishing (seen by the D1 -> A2
+    // converters) frees its tile; the last stage 2 of a batch finishing (seen
+    // by the epilogue) frees its D1/A2 region.  The MMA thread only commits
+    // D1FULL (once per batch) and D2FULL (once per group).
     if (warp == 0) {
         // ---------------- TMA producer: one batch tile per slot ----------------
-        if (lane == 0) {
-            int64_t issued = 0;
-            for (int64_t j = 0; j < nb; ++j) {
-                const int s = int(j % C::SX);
-                if (!wait_bounded(bar(C::EMPTY + s), uint32_t((j / C::SX) & 1) ^ 1u, s_abort,
-                                  kSiteProducer, kWaitLimitNs, false))
-                    break;
-                const int64_t g0 = (blockIdx.x + j * gridDim.x) * int64_t(C::GB);
-                mbar_arrive_expect_tx(bar(C::FULL + s), C::XTILE);
-                const uint32_t dst = sbase + C::OFF_RAW + s * C::XTILE;
+        // The whole warp runs the loop (converged); one elected lane issues.
+        Ring rx;
+        uint32_t issued = 0;
+        int64_t g0 = int64_t(blockIdx.x) * C::GB;
+        const int64_t gstep = int64_t(gridDim.x) * C::GB;
+        for (int64_t j = 0; j < nb; ++j, g0 += gstep, rx.next(C::SX)) {
+            const bool ok = wait_bounded(bar(C::EMPTY + rx.idx), rx.phase ^ 1u, s_abort, kSiteProducer,
+                                         kWaitLimitNs, false);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(bar(C::FULL + rx.idx), C::XTILE);
+                const uint32_t dst = sbase + C::OFF_RAW + rx.idx * C::XTILE;
 #pragma unroll
                 for (int gp = 0; gp < C::GB; ++gp) {
 #pragma unroll
@@ -290,105 +310,99 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         const int xc = (N2 == 128) ? 64 * c : 0;
                         const int64_t row = (N2 == 128) ? g * N1 : (2 * g + c) * N1;
                         tma_load_2d(dst + c * C::CHUNK + gp * (N1 * 128), &tmap_x, xc, int(row),
-                                    bar(C::FULL + s));
+                                    bar(C::FULL + rx.idx));
                     }
                 }
-                issued = j + 1;
             }
-            // Drain: the last load issued into each slot has landed.
-            for (int s = 0; s < C::SX; ++s) {
-                if (issued > s) {
-                    const int64_t last = s + ((issued - 1 - s) / C::SX) * C::SX;
-                    wait_bounded(bar(C::FULL + s), uint32_t((last / C::SX) & 1), s_abort, kSiteDrain,
-                                 kWaitLimitNs, true);
-                }
-            }
+            __syncwarp();
+            ++issued;
         }
+        // Drain: every load issued has landed (the slots' last phases completed).
+        Ring rd;
+        for (uint32_t i = 0; i < issued; ++i, rd.next(C::SX))
+            if (i + C::SX >= issued)
+                wait_bounded(bar(C::FULL + rd.idx), rd.phase, s_abort, kSiteDrain, kWaitLimitNs, true);
+        __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            constexpr uint32_t idesc1 = idesc_bf16_f32(128, C::NS1);
-            constexpr uint32_t idesc2 = idesc_bf16_f32(128, N1);
-            const uint32_t a1s = sbase + C::OFF_A1, b2 = sbase + C::OFF_B2;
-            for (int64_t j = 0; j <= nb; ++j) {
-                if (j < nb) {  // stage 1 of batch j
-                    const int b = int(j % C::NB1);
-                    if (!wait_bounded(bar(C::D1EMPTY + b), uint32_t((j / C::NB1) & 1) ^ 1u, s_abort,
-                                      kSiteMma, kWaitLimitNs, false))
-                        break;
-                    uint32_t src0, src1, release;
-                    if (SCALED) {
-                        const int c2 = int(j % C::SC);
-                        if (!wait_bounded(bar(C::CFULL + c2), uint32_t((j / C::SC) & 1), s_abort, kSiteMma,
-                                          kWaitLimitNs, false))
-                            break;
-                        src0 = sbase + C::OFF_CONV + c2 * 2 * C::XTILE;
-                        src1 = src0 + C::XTILE;
-                        release = bar(C::CEMPTY + c2);
-                    } else {
-                        const int s = int(j % C::SX);
-                        if (!wait_bounded(bar(C::FULL + s), uint32_t((j / C::SX) & 1), s_abort, kSiteMma,
-                                          kWaitLimitNs, false))
-                            break;
-                        src0 = src1 = sbase + C::OFF_RAW + s * C::XTILE;
-                        release = bar(C::EMPTY + s);
-                    }
-                    tc_fence_after();
-                    const uint32_t d1 = tmem + C::R1(b);
+        // The whole warp runs the loop and the waits (converged, so every
+        // operand is warp-uniform); one elected lane issues MMAs and commits.
+        constexpr uint32_t idesc1 = idesc_bf16_f32(128, C::NS1);
+        constexpr uint32_t idesc2 = idesc_bf16_f32(128, N1);
+        const uint64_t b2d = sdesc_kmajor_sw128(sbase + C::OFF_B2);
+        const uint64_t a1d = sdesc_kmajor_sw128(sbase + C::OFF_A1);
+        // descriptor start addresses are in 16-byte units in the low bits
+        auto koff1 = [](int kk) { return uint64_t(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4); };
+        auto koff2 = [](int kk) { return uint64_t(((kk >> 2) * (N1 * 128) + (kk & 3) * 32) >> 4); };
+        Ring rin, r1, r1p, r2;  // input tiles, D1/A2 regions (stage 1 / stage 2), D2 regions
+        for (int64_t j = 0; j <= nb; ++j) {
+            if (j < nb) {  // stage 1 of batch j
+                bool ok = wait_bounded(bar(C::D1EMPTY + r1.idx), r1.phase ^ 1u, s_abort, kSiteMma, kWaitLimitNs,
+                                       false);
+                uint32_t src;
+                if (SCALED) {
+                    ok = ok && wait_bounded(bar(C::CFULL + rin.idx), rin.phase, s_abort, kSiteMma, kWaitLimitNs,
+                                            false);
+                    src = sbase + C::OFF_CONV + rin.idx * 2 * C::XTILE;
+                } else {
+                    ok = ok && wait_bounded(bar(C::FULL + rin.idx), rin.phase, s_abort, kSiteMma, kWaitLimitNs,
+                                            false);
+                    src = sbase + C::OFF_RAW + rin.idx * C::XTILE;
+                }
+                if (!__all_sync(0xffffffffu, ok)) break;
+                tc_fence_after();
+                const uint32_t d1 = tmem + C::R1(int(r1.idx));
+                const uint64_t bd = sdesc_kmajor_sw128(src);
+                if (elect_one()) {
 #pragma unroll
                     for (int pass = 0; pass < (SCALED ? 2 : 1); ++pass) {
-                        const uint32_t src = pass ? src1 : src0;
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t off = uint32_t((kk & 3) * 32);
-                            const uint64_t bd = sdesc_kmajor_sw128(src + (kk >> 2) * C::CHUNK + off);
+                            const uint64_t b = bd + koff1(kk) + uint64_t(pass * (C::XTILE >> 4));
                             if (C::A1_TMEM)
-                                mma_ts(d1, tmem + 8 * kk, bd, idesc1, (pass | kk) != 0);
+                                mma_ts(d1, tmem + 8 * kk, b, idesc1, (pass | kk) != 0);
                             else
-                                mma_ss(d1, sdesc_kmajor_sw128(a1s + (kk >> 2) * 16384 + off), bd, idesc1,
+                                mma_ss(d1, a1d + uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), b, idesc1,
                                        (pass | kk) != 0);
                         }
                     }
-                    tc_commit(release);
-                    tc_commit(bar(C::D1FULL + b));
+                    tc_commit(bar(C::D1FULL + r1.idx));
                 }
-                if (j >= 1) {  // stage 2 of every group of batch j - 1
-                    const int64_t jp = j - 1;
-                    const int b = int(jp % C::NB1);
-                    if (!wait_bounded(bar(C::A2FULL + b), uint32_t((jp / C::NB1) & 1), s_abort, kSiteMma,
-                                      kWaitLimitNs, false))
-                        break;
-                    bool ok = true;
-#pragma unroll 1
-                    for (int gp = 0; gp < C::GB; ++gp) {
-                        const int64_t gi = jp * C::GB + gp;  // this CTA's group counter
-                        const int b2i = int(gi % C::NB2);
-                        if (!wait_bounded(bar(C::D2EMPTY + b2i), uint32_t((gi / C::NB2) & 1) ^ 1u, s_abort,
-                                          kSiteMma, kWaitLimitNs, false)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t d2 = tmem + C::R2(b2i), a2 = tmem + C::R1(b) + gp * N1;
-#pragma unroll
-                        for (int pass = 0; pass < 2; ++pass) {
-#pragma unroll
-                            for (int kk = 0; kk < N1 / 16; ++kk) {
-                                const uint64_t bd =
-                                    sdesc_kmajor_sw128(b2 + (kk >> 2) * (N1 * 128) + (kk & 3) * 32);
-                                mma_ts(d2, a2 + 16 * kk + 8 * pass, bd, idesc2, (pass | kk) != 0);
-                            }
-                        }
-                        tc_commit(bar(C::D2FULL + b2i));
-                    }
-                    if (!ok) break;
-                    tc_commit(bar(C::D1EMPTY + b));
-                }
+                __syncwarp();
+                rin.next(SCALED ? C::SC : C::SX);
+                r1.next(C::NB1);
             }
-            // Every MMA this thread issued has completed before TMEM is freed.
-            tc_commit(bar(C::TEARDOWN));
-            wait_bounded(bar(C::TEARDOWN), 0u, s_abort, kSiteDrain, kWaitLimitNs, true);
+            if (j >= 1) {  // stage 2 of every group of batch j - 1
+                bool ok = wait_bounded(bar(C::A2FULL + r1p.idx), r1p.phase, s_abort, kSiteMma, kWaitLimitNs, false);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                const uint32_t a2b = tmem + C::R1(int(r1p.idx));
+#pragma unroll
+                for (int gp = 0; gp < C::GB; ++gp) {
+                    ok = __all_sync(0xffffffffu, wait_bounded(bar(C::D2EMPTY + r2.idx), r2.phase ^ 1u, s_abort,
+                                                              kSiteMma, kWaitLimitNs, false));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t d2 = tmem + C::R2(int(r2.idx)), a2 = a2b + gp * N1;
+                    if (elect_one()) {
+#pragma unroll
+                        for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+                            for (int kk = 0; kk < N1 / 16; ++kk)
+                                mma_ts(d2, a2 + 16 * kk + 8 * pass, b2d + koff2(kk), idesc2, (pass | kk) != 0);
+                        tc_commit(bar(C::D2FULL + r2.idx));
+                    }
+                    __syncwarp();
+                    r2.next(C::NB2);
+                }
+                if (!ok) break;
+                r1p.next(C::NB1);
+            }
         }
+        // Every MMA this warp issued has completed before TMEM is freed.
+        if (elect_one()) tc_commit(bar(C::TEARDOWN));
+        __syncwarp();
+        wait_bounded(bar(C::TEARDOWN), 0u, s_abort, kSiteDrain, kWaitLimitNs, true);
+        __syncwarp();
     } else if (warp >= 4 && warp < 8) {
         // ---------------- x' = x * cinv -> hi / lo bf16 tiles ----------------
         if (SCALED) {
@@ -406,15 +420,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     cv[u][p] = uint64_t(__float_as_uint(cinv[r * N2 + b0 + 2 * p])) |
                                (uint64_t(__float_as_uint(cinv[r * N2 + b0 + 2 * p + 1])) << 32);
             }
-            for (int64_t j = 0; j < nb; ++j) {
-                const int s = int(j % C::SX), c2 = int(j % C::SC);
-                bool ok = wait_bounded(bar(C::FULL + s), uint32_t((j / C::SX) & 1), s_abort, kSiteXSplit,
-                                       kWaitLimitNs, false);
-                ok = ok && wait_bounded(bar(C::CEMPTY + c2), uint32_t((j / C::SC) & 1) ^ 1u, s_abort,
-                                        kSiteXSplit, kWaitLimitNs, false);
+            Ring rx, rc;
+            for (int64_t j = 0; j < nb; ++j, rx.next(C::SX), rc.next(C::SC)) {
+                bool ok = wait_bounded(bar(C::FULL + rx.idx), rx.phase, s_abort, kSiteXSplit, kWaitLimitNs, false);
+                ok = ok && wait_bounded(bar(C::CEMPTY + rc.idx), rc.phase ^ 1u, s_abort, kSiteXSplit,
+                                        kWaitLimitNs, false);
                 if (!__all_sync(0xffffffffu, ok)) break;  // the warp leaves together
-                const unsigned char *raw = smem + C::OFF_RAW + s * C::XTILE;
-                unsigned char *hi = smem + C::OFF_CONV + c2 * 2 * C::XTILE;
+                const unsigned char *raw = smem + C::OFF_RAW + rx.idx * C::XTILE;
+                unsigned char *hi = smem + C::OFF_CONV + rc.idx * 2 * C::XTILE;
                 unsigned char *lo = hi + C::XTILE;
 #pragma unroll
                 for (int gp = 0; gp < C::GB; ++gp) {
@@ -436,21 +449,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                 }
                 fence_proxy_async_smem();
-                mbar_arrive(bar(C::EMPTY + s));
-                mbar_arrive(bar(C::CFULL + c2));
+                mbar_arrive(bar(C::EMPTY + rx.idx));
+                mbar_arrive(bar(C::CFULL + rc.idx));
             }
         }
     } else if (warp >= 8 && warp < 12) {
         // ---------------- D1 (fp32) -> A2 (hi, lo bf16) in TMEM ----------------
         const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
-        for (int64_t j = 0; j < nb; ++j) {
-            const int b = int(j % C::NB1);
-            const bool ok = wait_bounded(bar(C::D1FULL + b), uint32_t((j / C::NB1) & 1), s_abort,
-                                         kSiteConvert, kWaitLimitNs, false);
+        Ring r1, rin;
+        for (int64_t j = 0; j < nb; ++j, r1.next(C::NB1), rin.next(SCALED ? C::SC : C::SX)) {
+            const bool ok = wait_bounded(bar(C::D1FULL + r1.idx), r1.phase, s_abort, kSiteConvert, kWaitLimitNs,
+                                         false);
             // reconverge before the warp-collective TMEM loads; leave together
             if (!__all_sync(0xffffffffu, ok)) break;
+            // stage 1 of batch j is done: its input tile may be refilled
+            mbar_arrive(bar((SCALED ? C::CEMPTY : C::EMPTY) + rin.idx));
             tc_fence_after();
-            const uint32_t col0 = tmem + lane_off + C::R1(b);
+            const uint32_t col0 = tmem + lane_off + C::R1(int(r1.idx));
             constexpr int NK = C::NS1 / 16;
             constexpr int BATCH = NK < 4 ? NK : 4;
 #pragma unroll
@@ -474,90 +489,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(C::A2FULL + b));
+            mbar_arrive(bar(C::A2FULL + r1.idx));
         }
     } else if (warp >= 12) {
         // ---------------- epilogue: absmax, quantise, pack, store ----------------
+        // Each thread reads two TMEM lanes (16x256b): lane g8 (even output
+        // column) and lane g8 + 8 (odd column) of its 16-lane half, so both
+        // nibbles of every byte it writes are in its registers.
         const int q = warp & 3;
         const int et = tid - 384;
         const int tok_h = (32 * q) / N2;
         const int g8 = lane >> 2, qq = lane & 3;
-        const uint32_t lane_off = uint32_t(32 * q) << 16;
-        unsigned char *stg = smem + C::OFF_STG;
         constexpr int NK = N1 / 16;
+        constexpr bool ONE_PASS = N1 <= 64;  // all of a thread's values fit in registers
+        constexpr int V16_ROW = N2 / 32;     // 16-byte chunks per output row
+        constexpr int V16 = C::H * N1 * V16_ROW;
         const int64_t ng = nb * C::GB;
-        for (int64_t gi = 0; gi < ng; ++gi) {
-            const int b = int(gi % C::NB2);
-            const int64_t g = (blockIdx.x + (gi / C::GB) * gridDim.x) * int64_t(C::GB) + gi % C::GB;
-            const bool ok = wait_bounded(bar(C::D2FULL + b), uint32_t((gi / C::NB2) & 1), s_abort,
-                                         kSiteEpilogue, kWaitLimitNs, false);
-            // All four warps leave together, so none is left behind in a named barrier.
-            const bool warp_ok = __all_sync(0xffffffffu, ok);
-            if (named_barrier_any(1, 128, !warp_ok)) break;
-            __syncwarp();
-            tc_fence_after();
-            // pass 1: absmax over this warp's 32 lanes and all n1 columns (tree of maxima)
-            float mx4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            constexpr int BATCH = NK < 4 ? NK : 4;
-#pragma unroll
-            for (int k0 = 0; k0 < NK; k0 += BATCH) {
-                uint32_t v[BATCH][16];
-#pragma unroll
-                for (int r = 0; r < BATCH; ++r)
-                    if (k0 + r < NK) tmem_ld_32x32b_x16(tmem + lane_off + C::R2(b) + 16 * (k0 + r), v[r]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int r = 0; r < BATCH; ++r)
-                    if (k0 + r < NK)
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            mx4[e & 3] = fmaxf(mx4[e & 3], fabsf(__uint_as_float(v[r][e])));
-            }
-            float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            if (lane == 0) s_red[q] = mx;
-            named_barrier_sync(1, 128);  // maxima visible; the previous group's copy-out is done
-            float m = 0.0f;
-#pragma unroll
-            for (int w = 0; w < 4; ++w)
-                if ((32 * w) / N2 == tok_h) m = fmaxf(m, s_red[w]);
-            const float s = alpha * m / 7.0f;
-            const float inv = s > 0.0f ? fminf(1.0f / s, 3.0e38f) : 0.0f;
-            // pass 2: codes; thread holds lanes g8 (even column) and g8 + 8 (odd column)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int L0 = 32 * q + 16 * hf;
-                const int col_byte = 8 * ((L0 % N2) / 16) + g8;
-                const uint32_t taddr = tmem + (uint32_t(L0) << 16) + C::R2(b);
-                uint32_t r[NK][8];
-#pragma unroll
-                for (int cc = 0; cc < NK; ++cc) tmem_ld_16x256b_x2(taddr + 16 * cc, r[cc]);
-                tmem_wait_ld();
-                if (hf == 1) {  // every TMEM read of this group is done
-                    tc_fence_before();
-                    mbar_arrive(bar(C::D2EMPTY + b));
-                }
-                unsigned char *rowbase = stg + (tok_h * N1) * C::RS + col_byte;
-#pragma unroll
-                for (int cc = 0; cc < NK; ++cc) {
-#pragma unroll
-                    for (int rep = 0; rep < 2; ++rep) {
-                        const int i0 = 16 * cc + 8 * rep + 2 * qq;
-                        const uint32_t *rr = &r[cc][4 * rep];
-                        // byte(i0) = even | odd << 4, byte(i0 + 1) likewise; saturate to [-8, 7]
-                        const uint32_t w0 = pack_s4x2(round_code(rr[2], inv), round_code(rr[0], inv), 0u);
-                        const uint32_t w1 = pack_s4x2(round_code(rr[3], inv), round_code(rr[1], inv), w0);
-                        rowbase[i0 * C::RS] = uint8_t(w1 >> 8);
-                        rowbase[(i0 + 1) * C::RS] = uint8_t(w1);
-                    }
-                }
-            }
-            named_barrier_sync(1, 128);  // staging rows complete
-            const int64_t tok0 = C::H * g;
+        auto copy_out = [&](int64_t gprev, int buf) {
+            const int64_t tok0 = C::H * gprev;
             const int64_t valid = (T - tok0) < C::H ? (T - tok0) : C::H;
-            constexpr int V16_ROW = N2 / 32;           // 16-byte chunks per output row
-            constexpr int V16 = C::H * N1 * V16_ROW;    // per group
+            const unsigned char *st = smem + C::OFF_STG + buf * C::STG;
             uint8_t *gout = q_out + tok0 * (C::N / 2);
 #pragma unroll
             for (int e0 = 0; e0 < V16; e0 += 128) {
@@ -566,11 +517,124 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const int row = e / V16_ROW, c16 = e % V16_ROW;
                     if (row < valid * N1)
                         *reinterpret_cast<uint4 *>(gout + row * (N2 / 2) + 16 * c16) =
-                            *reinterpret_cast<const uint4 *>(stg + row * C::RS + 16 * c16);
+                            *reinterpret_cast<const uint4 *>(st + row * C::RS + 16 * c16);
                 }
             }
+        };
+        int64_t g_prev = -1;
+        Ring r2, r1;
+        int gp = 0;
+        int64_t g = int64_t(blockIdx.x) * C::GB;
+        const int64_t gskip = (int64_t(gridDim.x) - 1) * C::GB;  // jump to this CTA's next batch
+        for (int64_t gi = 0; gi < ng; ++gi) {
+            const int b = int(r2.idx);
+            const int buf = int(gi & 1);
+            const bool ok = wait_bounded(bar(C::D2FULL + b), r2.phase, s_abort, kSiteEpilogue, kWaitLimitNs, false);
+            // All four warps leave together, so none is left behind in a named barrier.
+            const bool warp_ok = __all_sync(0xffffffffu, ok);
+            if (named_barrier_any(1, 128, !warp_ok)) break;
+            __syncwarp();
+            if (gp == C::GB - 1) {
+                // every stage-2 MMA of this batch is done: its D1/A2 region may be reused
+                mbar_arrive(bar(C::D1EMPTY + r1.idx));
+                r1.next(C::NB1);
+            }
+            tc_fence_after();
+            uint32_t r[ONE_PASS ? 2 : 1][NK][8];
+            float mx4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            if (ONE_PASS) {
+#pragma unroll
+                for (int hf = 0; hf < (ONE_PASS ? 2 : 1); ++hf)
+#pragma unroll
+                    for (int cc = 0; cc < NK; ++cc)
+                        tmem_ld_16x256b_x2(tmem + (uint32_t(32 * q + 16 * hf) << 16) + C::R2(b) + 16 * cc,
+                                           r[hf][cc]);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar(C::D2EMPTY + b));  // D2 region free for the next stage 2
+#pragma unroll
+                for (int hf = 0; hf < (ONE_PASS ? 2 : 1); ++hf)
+#pragma unroll
+                    for (int cc = 0; cc < NK; ++cc)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            mx4[e & 3] = fmaxf(mx4[e & 3], fabsf(__uint_as_float(r[hf][cc][e])));
+            } else {
+                // absmax from a first read (32x32b, thread = lane) in batches of 64 columns
+                const uint32_t lane_off = uint32_t(32 * q) << 16;
+                constexpr int BATCH = NK < 4 ? NK : 4;
+#pragma unroll
+                for (int k0 = 0; k0 < NK; k0 += BATCH) {
+                    uint32_t v[BATCH][16];
+#pragma unroll
+                    for (int z = 0; z < BATCH; ++z)
+                        if (k0 + z < NK) tmem_ld_32x32b_x16(tmem + lane_off + C::R2(b) + 16 * (k0 + z), v[z]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int z = 0; z < BATCH; ++z)
+                        if (k0 + z < NK)
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                mx4[e & 3] = fmaxf(mx4[e & 3], fabsf(__uint_as_float(v[z][e])));
+                }
+            }
+            float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0) s_red[4 * buf + q] = mx;
+            // maxima visible; every thread finished writing the previous group's staging rows
+            named_barrier_sync(1, 128);
+            if (g_prev >= 0) copy_out(g_prev, buf ^ 1);
+            float m = 0.0f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                if ((32 * w) / N2 == tok_h) m = fmaxf(m, s_red[4 * buf + w]);
+            const float s = alpha * m / 7.0f;
+            const float inv = s > 0.0f ? fminf(1.0f / s, 3.0e38f) : 0.0f;
+            unsigned char *stg = smem + C::OFF_STG + buf * C::STG;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int L0 = 32 * q + 16 * hf;
+                const int col_byte = 8 * ((L0 % N2) / 16) + g8;
+                unsigned char *rowbase = stg + (tok_h * N1) * C::RS + col_byte;
+                uint32_t rl[NK][8];
+                if (!ONE_PASS) {
+#pragma unroll
+                    for (int cc = 0; cc < NK; ++cc)
+                        tmem_ld_16x256b_x2(tmem + (uint32_t(L0) << 16) + C::R2(b) + 16 * cc, rl[cc]);
+                    tmem_wait_ld();
+                    if (hf == 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar(C::D2EMPTY + b));
+                    }
+                }
+#pragma unroll
+                for (int cc = 0; cc < NK; ++cc) {
+#pragma unroll
+                    for (int rep = 0; rep < 2; ++rep) {
+                        const int i0 = 16 * cc + 8 * rep + 2 * qq;
+                        const uint32_t *rr = ONE_PASS ? &r[hf & (ONE_PASS ? 1 : 0)][cc][4 * rep] : &rl[cc][4 * rep];
+                        // byte(i0) = even | odd << 4, byte(i0 + 1) likewise; saturate to [-8, 7]
+                        const uint32_t w0 = pack_s4x2(round_code(rr[2], inv), round_code(rr[0], inv), 0u);
+                        const uint32_t w1 = pack_s4x2(round_code(rr[3], inv), round_code(rr[1], inv), w0);
+                        rowbase[i0 * C::RS] = uint8_t(w1 >> 8);
+                        rowbase[(i0 + 1) * C::RS] = uint8_t(w1);
+                    }
+                }
+            }
+            const int64_t tok0 = C::H * g;
             if (lane == 0 && (32 * q) % N2 == 0 && tok0 + tok_h < T) scale_out[tok0 + tok_h] = s;
+            g_prev = g;
+            r2.next(C::NB2);
+            if (++gp == C::GB) {
+                gp = 0;
+                g += gskip;
+            }
+            ++g;
         }
+        // the last group's rows: everyone has written them once all pass this barrier
+        named_barrier_sync(1, 128);
+        if (g_prev >= 0) copy_out(g_prev, int((ng - 1) & 1));
     }
 
     tc_fence_before();
