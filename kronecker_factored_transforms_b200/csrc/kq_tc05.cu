@@ -61,7 +61,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kTcThreads = 512;
+constexpr int kTcThreads = 640;  // 5 warpgroups, at most 96 registers per thread
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // about one second
 
 enum : unsigned {
@@ -128,14 +128,14 @@ struct Cfg {
     static constexpr int OFF_B2 = 0;
     static constexpr int OFF_A1 = align_up(OFF_B2 + NCH2 * N1 * 128, 1024);
     static constexpr int OFF_RAW = OFF_A1 + (A1_TMEM ? 0 : 32768);
-    static constexpr int FIXED = OFF_RAW + (SCALED ? SC * 2 * XTILE : 0) + 2 * STG + 2048;
+    static constexpr int FIXED = OFF_RAW + (SCALED ? SC * 2 * XTILE : 0) + 4 * STG + 2048;
     static constexpr int SX = imax(2, imin(8, (222 * 1024 - FIXED) / XTILE));  // raw x stages
     static constexpr int OFF_CONV = OFF_RAW + SX * XTILE;
     static constexpr int OFF_STG = OFF_CONV + (SCALED ? SC * 2 * XTILE : 0);
     static constexpr int NBAR = 2 * SX + 2 * SC + 3 * NB1 + 2 * NB2 + 1;
-    static constexpr int OFF_BAR = align_up(OFF_STG + 2 * STG, 16);  // two staging buffers
-    static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem base, abort flag, 2 x 4 maxima
-    static constexpr int SMEM = OFF_MISC + 48 + 1024;    // + slack for 1024-byte alignment
+    static constexpr int OFF_BAR = align_up(OFF_STG + 4 * STG, 16);  // 2 epilogues x 2 staging buffers
+    static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem base, abort flag, 2 x 2 x 4 maxima
+    static constexpr int SMEM = OFF_MISC + 80 + 1024;    // + slack for 1024-byte alignment
     // barrier indices
     static constexpr int FULL = 0, EMPTY = SX, CFULL = 2 * SX, CEMPTY = 2 * SX + SC;
     static constexpr int D1FULL = 2 * SX + 2 * SC, A2FULL = D1FULL + NB1, D1EMPTY = A2FULL + NB1;
@@ -283,7 +283,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-
     // Release of x tiles: stage 1 of a batch finishing (seen by the D1 -> A2
     // converters) frees its tile; the last stage 2 of a batch finishing (seen
     // by the epilogue) frees its D1/A2 region.  The MMA thread only commits
@@ -467,7 +466,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             const uint32_t col0 = tmem + lane_off + C::R1(int(r1.idx));
             constexpr int NK = C::NS1 / 16;
-            constexpr int BATCH = NK < 4 ? NK : 4;
+            constexpr int BATCH = NK < 2 ? NK : 2;
 #pragma unroll
             for (int k0 = 0; k0 < NK; k0 += BATCH) {
                 uint32_t v[BATCH][16];
@@ -493,22 +492,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp >= 12) {
         // ---------------- epilogue: absmax, quantise, pack, store ----------------
-        // Each thread reads two TMEM lanes (16x256b): lane g8 (even output
-        // column) and lane g8 + 8 (odd column) of its 16-lane half, so both
-        // nibbles of every byte it writes are in its registers.
+        // Two epilogue warpgroups take alternate groups.  Each thread reads two
+        // TMEM lanes (16x256b): lane g8 (even output column) and lane g8 + 8
+        // (odd column) of its 16-lane half, so both nibbles of every byte it
+        // writes are in its registers.
+        const int ew = (warp - 12) >> 2;  // which epilogue warpgroup
         const int q = warp & 3;
-        const int et = tid - 384;
+        const int et = tid - 384 - 128 * ew;
+        const uint32_t nbar = 1u + uint32_t(ew);
         const int tok_h = (32 * q) / N2;
         const int g8 = lane >> 2, qq = lane & 3;
+        float *red = s_red + 8 * ew;
         constexpr int NK = N1 / 16;
-        constexpr bool ONE_PASS = N1 <= 64;  // all of a thread's values fit in registers
+        constexpr bool ONE_PASS = false;  // re-read TMEM rather than hold a group in registers
         constexpr int V16_ROW = N2 / 32;     // 16-byte chunks per output row
         constexpr int V16 = C::H * N1 * V16_ROW;
-        const int64_t ng = nb * C::GB;
-        auto copy_out = [&](int64_t gprev, int buf) {
+        const uint32_t ng = uint32_t(nb) * C::GB;
+        auto copy_out = [&](int64_t gprev, int sb) {
             const int64_t tok0 = C::H * gprev;
             const int64_t valid = (T - tok0) < C::H ? (T - tok0) : C::H;
-            const unsigned char *st = smem + C::OFF_STG + buf * C::STG;
+            const unsigned char *st = smem + C::OFF_STG + sb * C::STG;
             uint8_t *gout = q_out + tok0 * (C::N / 2);
 #pragma unroll
             for (int e0 = 0; e0 < V16; e0 += 128) {
@@ -522,33 +525,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
         };
         int64_t g_prev = -1;
-        Ring r2, r1;
-        int gp = 0;
-        int64_t g = int64_t(blockIdx.x) * C::GB;
-        const int64_t gskip = (int64_t(gridDim.x) - 1) * C::GB;  // jump to this CTA's next batch
-        for (int64_t gi = 0; gi < ng; ++gi) {
-            const int b = int(r2.idx);
-            const int buf = int(gi & 1);
-            const bool ok = wait_bounded(bar(C::D2FULL + b), r2.phase, s_abort, kSiteEpilogue, kWaitLimitNs, false);
+        int it = 0;
+        for (uint32_t gi = uint32_t(ew); gi < ng; gi += 2, ++it) {
+            const uint32_t b = gi % C::NB2, ph = (gi / C::NB2) & 1u;
+            const uint32_t jb = gi / C::GB, gp = gi % C::GB;
+            const int64_t g = (int64_t(blockIdx.x) + int64_t(jb) * gridDim.x) * C::GB + gp;
+            const int buf = it & 1;
+            const bool ok = wait_bounded(bar(C::D2FULL + b), ph, s_abort, kSiteEpilogue, kWaitLimitNs, false);
             // All four warps leave together, so none is left behind in a named barrier.
             const bool warp_ok = __all_sync(0xffffffffu, ok);
-            if (named_barrier_any(1, 128, !warp_ok)) break;
+            if (named_barrier_any(nbar, 128, !warp_ok)) break;
             __syncwarp();
             if (gp == C::GB - 1) {
                 // every stage-2 MMA of this batch is done: its D1/A2 region may be reused
-                mbar_arrive(bar(C::D1EMPTY + r1.idx));
-                r1.next(C::NB1);
+                mbar_arrive(bar(C::D1EMPTY + int(jb % C::NB1)));
             }
             tc_fence_after();
             uint32_t r[ONE_PASS ? 2 : 1][NK][8];
             float mx4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             if (ONE_PASS) {
 #pragma unroll
-                for (int hf = 0; hf < (ONE_PASS ? 2 : 1); ++hf)
+                for (int hf = 0; hf < (ONE_PASS ? 2 : 1); ++hf) {
+                    const uint32_t taddr = tmem + (uint32_t(32 * q + 16 * hf) << 16) + C::R2(int(b));
+                    if (N1 == 64)
+                        tmem_ld_16x256b_x8(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[hf][0][0]));
+                    else
 #pragma unroll
-                    for (int cc = 0; cc < NK; ++cc)
-                        tmem_ld_16x256b_x2(tmem + (uint32_t(32 * q + 16 * hf) << 16) + C::R2(b) + 16 * cc,
-                                           r[hf][cc]);
+                        for (int cc = 0; cc < NK; ++cc) tmem_ld_16x256b_x2(taddr + 16 * cc, r[hf][cc]);
+                }
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(bar(C::D2EMPTY + b));  // D2 region free for the next stage 2
@@ -560,15 +564,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         for (int e = 0; e < 8; ++e)
                             mx4[e & 3] = fmaxf(mx4[e & 3], fabsf(__uint_as_float(r[hf][cc][e])));
             } else {
-                // absmax from a first read (32x32b, thread = lane) in batches of 64 columns
+                // absmax from a first read (32x32b, thread = lane) in batches of 32 columns
                 const uint32_t lane_off = uint32_t(32 * q) << 16;
-                constexpr int BATCH = NK < 4 ? NK : 4;
+                constexpr int BATCH = NK < 2 ? NK : 2;
 #pragma unroll
                 for (int k0 = 0; k0 < NK; k0 += BATCH) {
                     uint32_t v[BATCH][16];
 #pragma unroll
                     for (int z = 0; z < BATCH; ++z)
-                        if (k0 + z < NK) tmem_ld_32x32b_x16(tmem + lane_off + C::R2(b) + 16 * (k0 + z), v[z]);
+                        if (k0 + z < NK) tmem_ld_32x32b_x16(tmem + lane_off + C::R2(int(b)) + 16 * (k0 + z), v[z]);
                     tmem_wait_ld();
 #pragma unroll
                     for (int z = 0; z < BATCH; ++z)
@@ -581,17 +585,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            if (lane == 0) s_red[4 * buf + q] = mx;
-            // maxima visible; every thread finished writing the previous group's staging rows
-            named_barrier_sync(1, 128);
-            if (g_prev >= 0) copy_out(g_prev, buf ^ 1);
+            if (lane == 0) red[4 * buf + q] = mx;
+            // maxima visible; every thread finished writing its previous group's staging rows
+            named_barrier_sync(nbar, 128);
+            if (g_prev >= 0) copy_out(g_prev, 2 * ew + (buf ^ 1));
             float m = 0.0f;
 #pragma unroll
             for (int w = 0; w < 4; ++w)
-                if ((32 * w) / N2 == tok_h) m = fmaxf(m, s_red[4 * buf + w]);
+                if ((32 * w) / N2 == tok_h) m = fmaxf(m, red[4 * buf + w]);
             const float s = alpha * m / 7.0f;
             const float inv = s > 0.0f ? fminf(1.0f / s, 3.0e38f) : 0.0f;
-            unsigned char *stg = smem + C::OFF_STG + buf * C::STG;
+            unsigned char *stg = smem + C::OFF_STG + (2 * ew + buf) * C::STG;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const int L0 = 32 * q + 16 * hf;
@@ -601,7 +605,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!ONE_PASS) {
 #pragma unroll
                     for (int cc = 0; cc < NK; ++cc)
-                        tmem_ld_16x256b_x2(tmem + (uint32_t(L0) << 16) + C::R2(b) + 16 * cc, rl[cc]);
+                        tmem_ld_16x256b_x2(tmem + (uint32_t(L0) << 16) + C::R2(int(b)) + 16 * cc, rl[cc]);
                     tmem_wait_ld();
                     if (hf == 1) {
                         tc_fence_before();
@@ -625,16 +629,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int64_t tok0 = C::H * g;
             if (lane == 0 && (32 * q) % N2 == 0 && tok0 + tok_h < T) scale_out[tok0 + tok_h] = s;
             g_prev = g;
-            r2.next(C::NB2);
-            if (++gp == C::GB) {
-                gp = 0;
-                g += gskip;
-            }
-            ++g;
         }
         // the last group's rows: everyone has written them once all pass this barrier
-        named_barrier_sync(1, 128);
-        if (g_prev >= 0) copy_out(g_prev, int((ng - 1) & 1));
+        named_barrier_sync(nbar, 128);
+        if (g_prev >= 0) copy_out(g_prev, 2 * ew + ((it - 1) & 1));
     }
 
     tc_fence_before();
