@@ -164,18 +164,17 @@ __device__ __forceinline__ uint16_t a1_value(const uint16_t *__restrict__ P2, in
     return (h == hk) ? P2[b * N2 + j] : uint16_t(0);
 }
 
-// v = hi + lo with hi = v truncated to bf16 (its top 16 bits) and lo = v - hi
-// (exact in fp32), then lo rounded to bf16 to nearest (ties away from zero,
-// by adding half an ulp to the magnitude bits): about 16 significant bits in
-// all, using only integer and fp32 pipes.  Takes two fp32 values as one
-// 64-bit pair; returns the two hi values packed (first in the low half) and
-// the two lo ones.
+// v = hi + lo with hi = v truncated to bf16 (its top 16 bits, a byte permute)
+// and lo = v - hi (exact in fp32) rounded to bf16 (one conversion per pair):
+// about 16 significant bits in all.  Takes two fp32 values as one 64-bit
+// pair; returns the two hi values packed (first in the low half) and the two
+// lo ones.
 __device__ __forceinline__ void split2(uint64_t v, uint32_t &hi, uint32_t &lo) {
     const uint32_t v0 = uint32_t(v), v1 = uint32_t(v >> 32);
     const uint64_t t = uint64_t(v0 & 0xFFFF0000u) | (uint64_t(v1 & 0xFFFF0000u) << 32);
     const uint64_t l = f32x2_sub(v, t);
     hi = __byte_perm(v0, v1, 0x7632);
-    lo = __byte_perm(uint32_t(l) + 0x8000u, uint32_t(l >> 32) + 0x8000u, 0x7632);
+    lo = pack_bf16x2(__uint_as_float(uint32_t(l)), __uint_as_float(uint32_t(l >> 32)));
 }
 
 // round_half_even(y * inv) as an int, valid for |y * inv| < 2^22 (alpha >= 2^-19):
