@@ -27,9 +27,9 @@
 // k - 2 is issued after stage 1 of group k and the tensor pipe never waits
 // for work the issuer has just queued.
 //
-// Warp roles: 0 TMA producer | 1 TMEM allocator + MMA issuer | 4-7 x' split
-// (cinv only) | 8-11 P2^T into TMEM, then D1 -> A2 conversion | 12-15
-// epilogue.  Every mbarrier wait is bounded: after about a second it ORs a
+// Warp roles: 0 TMA producer | 1 TMEM allocator + MMA issuer | 2-7, 20-21 x'
+// split (cinv only) | 8-11 P2^T into TMEM, then D1 -> A2 conversion | 12-15
+// and 16-19 two epilogue warpgroups taking alternate groups.  Every mbarrier wait is bounded: after about a second it ORs a
 // site bit into g_device_error, raises a CTA-wide abort flag and the roles
 // drain and exit.
 #include <cuda.h>
@@ -61,7 +61,8 @@ namespace {
 
 using namespace tc;
 
-constexpr int kTcThreads = 640;  // 5 warpgroups, at most 96 registers per thread
+constexpr int kTcThreads = 704;  // 22 warps, at most 88 registers per thread
+constexpr int kXThreads = 256;   // x' split: warps 2-7 and 20-21
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // about one second
 
 enum : unsigned {
@@ -220,10 +221,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < C::SX; ++s) {
             mbar_init(bar(C::FULL + s), 1);
-            mbar_init(bar(C::EMPTY + s), 128);
+            mbar_init(bar(C::EMPTY + s), SCALED ? kXThreads : 128);
         }
         for (int c = 0; c < C::SC; ++c) {
-            mbar_init(bar(C::CFULL + c), 128);
+            mbar_init(bar(C::CFULL + c), kXThreads);
             mbar_init(bar(C::CEMPTY + c), 128);
         }
         for (int b = 0; b < C::NB1; ++b) {
@@ -401,16 +402,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
         wait_bounded(bar(C::TEARDOWN), 0u, s_abort, kSiteDrain, kWaitLimitNs, true);
         __syncwarp();
-    } else if (warp >= 4 && warp < 8) {
+    } else if ((warp >= 2 && warp < 8) || warp >= 20) {
         // ---------------- x' = x * cinv -> hi / lo bf16 tiles ----------------
         if (SCALED) {
-            const int t = tid - 128;
-            // thread t handles unit e = t + 128 u (u < n1/8) of every group of the batch;
-            // its cinv values depend only on (u, t)
-            uint64_t cv[N1 / 8][4];
+            const int t = warp < 8 ? tid - 64 : tid - 640 + 192;  // 0 .. kXThreads - 1
+            constexpr int UPT = 16 * N1 / kXThreads;             // units per thread per group
+            // thread t handles unit e = t + kXThreads u (u < UPT) of every group of the
+            // batch; its cinv values depend only on (u, t)
+            uint64_t cv[UPT][4];
 #pragma unroll
-            for (int u = 0; u < N1 / 8; ++u) {
-                const int e = t + 128 * u;
+            for (int u = 0; u < UPT; ++u) {
+                const int e = t + kXThreads * u;
                 const int c = e / (8 * N1), rem = e % (8 * N1), r = rem >> 3, up = rem & 7;
                 const int b0 = (N2 == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
 #pragma unroll
@@ -430,8 +432,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int gp = 0; gp < C::GB; ++gp) {
 #pragma unroll
-                    for (int u = 0; u < N1 / 8; ++u) {
-                        const int e = t + 128 * u;
+                    for (int u = 0; u < UPT; ++u) {
+                        const int e = t + kXThreads * u;
                         const int c = e / (8 * N1), rem = e % (8 * N1);
                         const int off = c * C::CHUNK + gp * (N1 * 128) + rem * 16;
                         const uint4 in = *reinterpret_cast<const uint4 *>(raw + off);
@@ -489,7 +491,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_before();
             mbar_arrive(bar(C::A2FULL + r1.idx));
         }
-    } else if (warp >= 12) {
+    } else if (warp >= 12 && warp < 20) {
         // ---------------- epilogue: absmax, quantise, pack, store ----------------
         // Two epilogue warpgroups take alternate groups.  Each thread reads two
         // TMEM lanes (16x256b): lane g8 (even output column) and lane g8 + 8
