@@ -21,8 +21,9 @@
 //   stage 2 (TS MMA)  D2[l][i]  = sum_a A2[l][a] * P1[a][i]   (A from TMEM)
 //   epilogue          absmax over the token's lanes, quantise, pack into a
 //                     bank-spread staging area, 16-byte stores to HBM.
-// With cinv, warps 4-7 first turn each raw x tile into x' = x * cinv split
-// into hi and lo bf16 tiles; stage 1 then accumulates both.  TMEM holds four
+// With cinv, the x' split warps turn each raw x tile into x' = x * cinv
+// split into a hi bf16 tile (written over x) and a lo bf16 tile; stage 1
+// then accumulates both.  TMEM holds four
 // D1/A2 regions and three D2 regions (n1 <= 64) so that stage 2 of group
 // k - 2 is issued after stage 1 of group k and the tensor pipe never waits
 // for work the issuer has just queued.
@@ -123,16 +124,16 @@ struct Cfg {
     static constexpr int NB2 = (A1COLS + NB1 * R1W + 3 * N1P <= 512) ? 3 : 2;  // D2 regions (groups)
     static constexpr int TMEM_USED = A1COLS + NB1 * R1W + NB2 * N1P;
     static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
-    static constexpr int SC = 2;                     // split x' tile stages (cinv)
+    static constexpr int SC = 2;                     // lo-half tile stages (cinv); hi is written in place
     static constexpr int RS = N2 / 2 + 16;           // staging row stride (bytes), bank-spread
     static constexpr int STG = H * N1 * RS;          // staging bytes per group
     static constexpr int OFF_B2 = 0;
     static constexpr int OFF_A1 = align_up(OFF_B2 + NCH2 * N1 * 128, 1024);
     static constexpr int OFF_RAW = OFF_A1 + (A1_TMEM ? 0 : 32768);
-    static constexpr int FIXED = OFF_RAW + (SCALED ? SC * 2 * XTILE : 0) + 4 * STG + 2048;
+    static constexpr int FIXED = OFF_RAW + (SCALED ? SC * XTILE : 0) + 4 * STG + 2048;
     static constexpr int SX = imax(2, imin(8, (222 * 1024 - FIXED) / XTILE));  // raw x stages
     static constexpr int OFF_CONV = OFF_RAW + SX * XTILE;
-    static constexpr int OFF_STG = OFF_CONV + (SCALED ? SC * 2 * XTILE : 0);
+    static constexpr int OFF_STG = OFF_CONV + (SCALED ? SC * XTILE : 0);
     static constexpr int NBAR = 2 * SX + 2 * SC + 3 * NB1 + 2 * NB2 + 1;
     static constexpr int OFF_BAR = align_up(OFF_STG + 4 * STG, 16);  // 2 epilogues x 2 staging buffers
     static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem base, abort flag, 2 x 2 x 4 maxima
@@ -221,16 +222,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < C::SX; ++s) {
             mbar_init(bar(C::FULL + s), 1);
-            mbar_init(bar(C::EMPTY + s), SCALED ? kXThreads : 128);
+            mbar_init(bar(C::EMPTY + s), 1);
         }
         for (int c = 0; c < C::SC; ++c) {
             mbar_init(bar(C::CFULL + c), kXThreads);
-            mbar_init(bar(C::CEMPTY + c), 128);
+            mbar_init(bar(C::CEMPTY + c), 1);
         }
         for (int b = 0; b < C::NB1; ++b) {
             mbar_init(bar(C::D1FULL + b), 1);
             mbar_init(bar(C::A2FULL + b), 128);
-            mbar_init(bar(C::D1EMPTY + b), 128);
+            mbar_init(bar(C::D1EMPTY + b), 1);
         }
         for (int b = 0; b < C::NB2; ++b) {
             mbar_init(bar(C::D2FULL + b), 1);
@@ -333,31 +334,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // descriptor start addresses are in 16-byte units in the low bits
         auto koff1 = [](int kk) { return uint64_t(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4); };
         auto koff2 = [](int kk) { return uint64_t(((kk >> 2) * (N1 * 128) + (kk & 3) * 32) >> 4); };
-        Ring rin, r1, r1p, r2;  // input tiles, D1/A2 regions (stage 1 / stage 2), D2 regions
+        Ring rin, rxs, r1, r1p, r2;  // input tiles, raw slots, D1/A2 regions (stage 1 / 2), D2 regions
         for (int64_t j = 0; j <= nb; ++j) {
             if (j < nb) {  // stage 1 of batch j
                 bool ok = wait_bounded(bar(C::D1EMPTY + r1.idx), r1.phase ^ 1u, s_abort, kSiteMma, kWaitLimitNs,
                                        false);
-                uint32_t src;
+                uint32_t src, src_lo;
                 if (SCALED) {
                     ok = ok && wait_bounded(bar(C::CFULL + rin.idx), rin.phase, s_abort, kSiteMma, kWaitLimitNs,
                                             false);
-                    src = sbase + C::OFF_CONV + rin.idx * 2 * C::XTILE;
+                    src = sbase + C::OFF_RAW + rxs.idx * C::XTILE;      // hi half, in place of x
+                    src_lo = sbase + C::OFF_CONV + rin.idx * C::XTILE;  // lo half
                 } else {
                     ok = ok && wait_bounded(bar(C::FULL + rin.idx), rin.phase, s_abort, kSiteMma, kWaitLimitNs,
                                             false);
-                    src = sbase + C::OFF_RAW + rin.idx * C::XTILE;
+                    src = src_lo = sbase + C::OFF_RAW + rin.idx * C::XTILE;
                 }
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
                 const uint32_t d1 = tmem + C::R1(int(r1.idx));
-                const uint64_t bd = sdesc_kmajor_sw128(src);
+                const uint64_t bd_hi = sdesc_kmajor_sw128(src), bd_lo = sdesc_kmajor_sw128(src_lo);
                 if (elect_one()) {
 #pragma unroll
                     for (int pass = 0; pass < (SCALED ? 2 : 1); ++pass) {
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t b = bd + koff1(kk) + uint64_t(pass * (C::XTILE >> 4));
+                            const uint64_t b = (pass ? bd_lo : bd_hi) + koff1(kk);
                             if (C::A1_TMEM)
                                 mma_ts(d1, tmem + 8 * kk, b, idesc1, (pass | kk) != 0);
                             else
@@ -365,10 +367,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                        (pass | kk) != 0);
                         }
                     }
+                    tc_commit(bar(C::EMPTY + rxs.idx));  // x (hi) tile slot free
+                    if (SCALED) tc_commit(bar(C::CEMPTY + rin.idx));  // lo tile free
                     tc_commit(bar(C::D1FULL + r1.idx));
                 }
                 __syncwarp();
                 rin.next(SCALED ? C::SC : C::SX);
+                rxs.next(C::SX);
                 r1.next(C::NB1);
             }
             if (j >= 1) {  // stage 2 of every group of batch j - 1
@@ -394,6 +399,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     r2.next(C::NB2);
                 }
                 if (!ok) break;
+                if (elect_one()) tc_commit(bar(C::D1EMPTY + r1p.idx));  // A2 region free
+                __syncwarp();
                 r1p.next(C::NB1);
             }
         }
@@ -426,9 +433,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 ok = ok && wait_bounded(bar(C::CEMPTY + rc.idx), rc.phase ^ 1u, s_abort, kSiteXSplit,
                                         kWaitLimitNs, false);
                 if (!__all_sync(0xffffffffu, ok)) break;  // the warp leaves together
-                const unsigned char *raw = smem + C::OFF_RAW + rx.idx * C::XTILE;
-                unsigned char *hi = smem + C::OFF_CONV + rc.idx * 2 * C::XTILE;
-                unsigned char *lo = hi + C::XTILE;
+                unsigned char *raw = smem + C::OFF_RAW + rx.idx * C::XTILE;  // x in, hi half out
+                unsigned char *lo = smem + C::OFF_CONV + rc.idx * C::XTILE;
 #pragma unroll
                 for (int gp = 0; gp < C::GB; ++gp) {
 #pragma unroll
@@ -444,26 +450,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             const uint64_t xv = uint64_t(w[p] << 16) | (uint64_t(w[p] & 0xFFFF0000u) << 32);
                             split2(f32x2_mul(xv, cv[u][p]), oh[p], ol[p]);
                         }
-                        *reinterpret_cast<uint4 *>(hi + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+                        *reinterpret_cast<uint4 *>(raw + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
                         *reinterpret_cast<uint4 *>(lo + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
                     }
                 }
                 fence_proxy_async_smem();
-                mbar_arrive(bar(C::EMPTY + rx.idx));
                 mbar_arrive(bar(C::CFULL + rc.idx));
             }
         }
     } else if (warp >= 8 && warp < 12) {
         // ---------------- D1 (fp32) -> A2 (hi, lo bf16) in TMEM ----------------
         const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
-        Ring r1, rin;
-        for (int64_t j = 0; j < nb; ++j, r1.next(C::NB1), rin.next(SCALED ? C::SC : C::SX)) {
+        Ring r1;
+        for (int64_t j = 0; j < nb; ++j, r1.next(C::NB1)) {
             const bool ok = wait_bounded(bar(C::D1FULL + r1.idx), r1.phase, s_abort, kSiteConvert, kWaitLimitNs,
                                          false);
             // reconverge before the warp-collective TMEM loads; leave together
             if (!__all_sync(0xffffffffu, ok)) break;
-            // stage 1 of batch j is done: its input tile may be refilled
-            mbar_arrive(bar((SCALED ? C::CEMPTY : C::EMPTY) + rin.idx));
             tc_fence_after();
             const uint32_t col0 = tmem + lane_off + C::R1(int(r1.idx));
             constexpr int NK = C::NS1 / 16;
@@ -505,7 +508,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int g8 = lane >> 2, qq = lane & 3;
         float *red = s_red + 8 * ew;
         constexpr int NK = N1 / 16;
-        constexpr bool ONE_PASS = false;  // re-read TMEM rather than hold a group in registers
+        constexpr bool ONE_PASS = false;  // re-read TMEM: a group does not fit in 80 registers
         constexpr int V16_ROW = N2 / 32;     // 16-byte chunks per output row
         constexpr int V16 = C::H * N1 * V16_ROW;
         const uint32_t ng = uint32_t(nb) * C::GB;
@@ -537,10 +540,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const bool warp_ok = __all_sync(0xffffffffu, ok);
             if (named_barrier_any(nbar, 128, !warp_ok)) break;
             __syncwarp();
-            if (gp == C::GB - 1) {
-                // every stage-2 MMA of this batch is done: its D1/A2 region may be reused
-                mbar_arrive(bar(C::D1EMPTY + int(jb % C::NB1)));
-            }
             tc_fence_after();
             uint32_t r[ONE_PASS ? 2 : 1][NK][8];
             float mx4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -565,28 +564,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         for (int e = 0; e < 8; ++e)
                             mx4[e & 3] = fmaxf(mx4[e & 3], fabsf(__uint_as_float(r[hf][cc][e])));
             } else {
-                // absmax from a first read (32x32b, thread = lane) in batches of 32 columns
+                // absmax from a first read (32x32b, thread = lane), 32 columns per load
                 const uint32_t lane_off = uint32_t(32 * q) << 16;
-                constexpr int BATCH = NK < 2 ? NK : 2;
+                if (N1 % 32 == 0) {
 #pragma unroll
-                for (int k0 = 0; k0 < NK; k0 += BATCH) {
-                    uint32_t v[BATCH][16];
+                    for (int k0 = 0; k0 < N1; k0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(tmem + lane_off + C::R2(int(b)) + k0, v);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int z = 0; z < BATCH; ++z)
-                        if (k0 + z < NK) tmem_ld_32x32b_x16(tmem + lane_off + C::R2(int(b)) + 16 * (k0 + z), v[z]);
-                    tmem_wait_ld();
+                        for (int e = 0; e < 32; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], fabsf(__uint_as_float(v[e])));
+                    }
+                } else {
 #pragma unroll
-                    for (int z = 0; z < BATCH; ++z)
-                        if (k0 + z < NK)
+                    for (int k0 = 0; k0 < NK; ++k0) {
+                        uint32_t v[16];
+                        tmem_ld_32x32b_x16(tmem + lane_off + C::R2(int(b)) + 16 * k0, v);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                mx4[e & 3] = fmaxf(mx4[e & 3], fabsf(__uint_as_float(v[z][e])));
+                        for (int e = 0; e < 16; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], fabsf(__uint_as_float(v[e])));
+                    }
                 }
             }
-            float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            if (lane == 0) red[4 * buf + q] = mx;
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            // non-negative floats order like their bit patterns: one warp reduction
+            const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
+            if (lane == 0) red[4 * buf + q] = __uint_as_float(wmax);
             // maxima visible; every thread finished writing its previous group's staging rows
             named_barrier_sync(nbar, 128);
             if (g_prev >= 0) copy_out(g_prev, 2 * ew + (buf ^ 1));
@@ -594,8 +597,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int w = 0; w < 4; ++w)
                 if ((32 * w) / N2 == tok_h) m = fmaxf(m, red[4 * buf + w]);
-            const float s = alpha * m / 7.0f;
-            const float inv = s > 0.0f ? fminf(1.0f / s, 3.0e38f) : 0.0f;
+            // s = alpha * max / 7 to within an ulp; codes use y * (1/s): both differ from the
+            // exact quotients by a few ulps, far inside the rounding-boundary window
+            const float s = alpha * m * (1.0f / 7.0f);
+            const float inv = s > 0.0f ? fminf(__fdividef(1.0f, s), 3.0e38f) : 0.0f;
             unsigned char *stg = smem + C::OFF_STG + (2 * ew + buf) * C::STG;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
@@ -604,9 +609,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 unsigned char *rowbase = stg + (tok_h * N1) * C::RS + col_byte;
                 uint32_t rl[NK][8];
                 if (!ONE_PASS) {
+                    if (N1 == 64)
+                        tmem_ld_16x256b_x8(tmem + (uint32_t(L0) << 16) + C::R2(int(b)),
+                                           *reinterpret_cast<uint32_t(*)[32]>(&rl[0][0]));
+                    else
 #pragma unroll
-                    for (int cc = 0; cc < NK; ++cc)
-                        tmem_ld_16x256b_x2(tmem + (uint32_t(L0) << 16) + C::R2(int(b)) + 16 * cc, rl[cc]);
+                        for (int cc = 0; cc < NK; ++cc)
+                            tmem_ld_16x256b_x2(tmem + (uint32_t(L0) << 16) + C::R2(int(b)) + 16 * cc, rl[cc]);
                     tmem_wait_ld();
                     if (hf == 1) {
                         tc_fence_before();
