@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="CPU time the reference arm's warm-up + timed steps aim at")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling runs)")
     return ap.parse_args()
@@ -98,6 +100,27 @@ def recorded_traffic(kernel_name):
 
 
 # ---------------------------------------------------------------------------
+# Multi-rank host logic: every rank owns one T-token shard; the step time is
+# the maximum over ranks and the value counts the tokens of all ranks.
+
+def max_over_ranks(x, device, world):
+    """Max of a per-rank float over the process group (identity when world == 1)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world, tokens_per_rank, steps, ms):
+    """Tokens processed by all ranks over ``steps`` steps, divided by the
+    slowest rank's elapsed time ``ms``."""
+    return world * tokens_per_rank * steps / (ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle timing (baseline leg and the reference arm).
 
 def time_oracle(w, seconds, max_tokens=None):
@@ -134,7 +157,7 @@ def run_reference(args):
     oracle.transform_quant(w.x[:probe], w.P1, w.P2, w.cinv, w.alpha, w.n1, w.n2, nthreads=nth,
                            want_codes=False)
     per_tok = (time.perf_counter() - t0) / probe
-    budget = 120.0 / max(1, args.steps + args.warmup)
+    budget = args.ref_seconds / max(1, args.steps + args.warmup)
     sample = int(max(1, min(w.T, budget / max(per_tok, 1e-9))))
     for _ in range(args.warmup):
         oracle.transform_quant(w.x[:sample], w.P1, w.P2, w.cinv, w.alpha, w.n1, w.n2, nthreads=nth,
@@ -282,11 +305,7 @@ def main():
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev, world)
     if _lib.kq_device_error(stream) != 0:
         raise RuntimeError("a bounded wait timed out inside the kernel")
 
@@ -326,10 +345,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev, world)
 
     clocks = sampler.report()
     if world > 1:
@@ -339,7 +355,7 @@ def main():
         return 0
 
     ms_step = ms / args.steps
-    value = world * T * args.steps / (ms / 1e3)
+    value = whole_job_tokens_per_s(world, T, args.steps, ms)
     hbm_peak, tf_peak, peak_kind = measured_peaks()
     bytes_launch = workload_bytes(T, n)
     flops_launch = workload_flops(T, n1, n2)
@@ -362,7 +378,7 @@ def main():
                                       "kernel": kernel}),
             "roofline": roof,
             "e2e": None if args.no_e2e else
-                   {"value": world * T * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+                   {"value": whole_job_tokens_per_s(world, T, args.e2e_steps, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps, "clocks": clocks}
     if world == 1 and not args.no_cpu_baseline:
