@@ -7,14 +7,16 @@
 // then per-token absmax, s = alpha * max / 7, round-half-even codes clamped
 // to [-8, 7], packed two per byte.  Only codes and scales reach HBM.
 //
-// Layout of the work (one CTA per SM, 16 warps, groups of H = 128 / n2
-// tokens so that the 128 TMEM lanes always hold 128 output columns):
-//   TMEM lane l = (h, m): token h of the group, output column j = pi(m) of
-//   its n2 columns.  pi interleaves each block of 16 columns (lanes 0-7 take
-//   the even columns, lanes 8-15 the odd ones) so that one thread of a
-//   16x256b TMEM load holds both nibbles of an output byte.
+// Layout of the work (one CTA per SM, 22 warps, groups of H = 128 / n2
+// tokens so that the 128 TMEM lanes always hold 128 output columns; stage 1
+// runs on batches of GB groups so that its MMAs are 128 wide):
+//   TMEM lane l = (h, m): token h of the group, output column
+//   j = lane_column(m) of its n2 columns.  Within each block of 32 lanes the
+//   columns are interleaved so that the thread of a 16x256b TMEM load that
+//   holds lanes g and g + 8 of both 16-lane halves holds four consecutive
+//   columns, i.e. two whole output bytes.
 //   stage 1           D1[l][a]  = sum_(h',b) A1[l][(h',b)] * X[a][(h',b)]
-//                     A1 = block-diag over h of P2^T (rows permuted by pi),
+//                     A1 = block-diag over h of P2^T (rows permuted as above),
 //                     resident in TMEM (or shared memory for n1 > 96);
 //                     X  = the group's x tile straight from TMA (K = 128).
 //   convert (TMEM)    D1 fp32 -> A2 = hi + lo bf16, in place, chunk by chunk.
@@ -23,16 +25,16 @@
 //                     bank-spread staging area, 16-byte stores to HBM.
 // With cinv, the x' split warps turn each raw x tile into x' = x * cinv
 // split into a hi bf16 tile (written over x) and a lo bf16 tile; stage 1
-// then accumulates both.  TMEM holds four
-// D1/A2 regions and three D2 regions (n1 <= 64) so that stage 2 of group
-// k - 2 is issued after stage 1 of group k and the tensor pipe never waits
-// for work the issuer has just queued.
+// then accumulates both.  TMEM holds P2^T, two D1/A2 regions (batches) and
+// three D2 regions (groups, n1 <= 64), so that stage 2 of batch k - 1 is
+// issued after stage 1 of batch k and the tensor pipe never waits for work
+// the issuer has just queued.
 //
 // Warp roles: 0 TMA producer | 1 TMEM allocator + MMA issuer | 2-7, 20-21 x'
 // split (cinv only) | 8-11 P2^T into TMEM, then D1 -> A2 conversion | 12-15
-// and 16-19 two epilogue warpgroups taking alternate groups.  Every mbarrier wait is bounded: after about a second it ORs a
-// site bit into g_device_error, raises a CTA-wide abort flag and the roles
-// drain and exit.
+// and 16-19 two epilogue warpgroups taking alternate groups.  Every mbarrier
+// wait is bounded: after about a second it ORs a site bit into
+// g_device_error, raises a CTA-wide abort flag and the roles drain and exit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -136,7 +138,7 @@ struct Cfg {
     static constexpr int OFF_STG = OFF_CONV + (SCALED ? SC * XTILE : 0);
     static constexpr int NBAR = 2 * SX + 2 * SC + 3 * NB1 + 2 * NB2 + 1;
     static constexpr int OFF_BAR = align_up(OFF_STG + 4 * STG, 16);  // 2 epilogues x 2 staging buffers
-    static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem base, abort flag, 2 x 2 x 4 maxima
+    static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem base, abort flag, the constant 1, 2 x 2 x 4 maxima
     static constexpr int SMEM = OFF_MISC + 80 + 1024;    // + slack for 1024-byte alignment
     // barrier indices
     static constexpr int FULL = 0, EMPTY = SX, CFULL = 2 * SX, CEMPTY = 2 * SX + SC;
@@ -157,13 +159,21 @@ __device__ __forceinline__ uint32_t swz128(int r, int k) {
     return uint32_t(r * 128 + ((((k >> 3) ^ (r & 7)) << 4) | ((k & 7) << 1)));
 }
 
-// Row l of A1 = block-diag over the stacked tokens of P2^T, rows permuted by pi:
-// A1[l][k] = P2[b][pi(m)] for l = (h, m), k = (h, b); zero off the diagonal blocks.
+// Output column held by TMEM lane m of a token (m < n2).  Within each block of
+// 32 lanes, lane 16 f + 8 s + g holds column 4 g + 2 f + s, so the thread
+// that a 16x256b load gives lanes g and g + 8 of both 16-lane halves holds
+// four consecutive columns: two whole bytes of every output row.
+__host__ __device__ constexpr int lane_column(int m) {
+    return (m & ~31) | ((m & 7) << 2) | (((m >> 4) & 1) << 1) | ((m >> 3) & 1);
+}
+
+// Row l of A1 = block-diag over the stacked tokens of P2^T, rows permuted:
+// A1[l][k] = P2[b][lane_column(m)] for l = (h, m), k = (h, b); zero off the
+// diagonal blocks.
 template <int N2>
 __device__ __forceinline__ uint16_t a1_value(const uint16_t *__restrict__ P2, int l, int k) {
     const int h = l / N2, m = l % N2, hk = k / N2, b = k % N2;
-    const int j = (m & ~15) | ((m & 7) << 1) | ((m >> 3) & 1);
-    return (h == hk) ? P2[b * N2 + j] : uint16_t(0);
+    return (h == hk) ? P2[b * N2 + lane_column(m)] : uint16_t(0);
 }
 
 // v = hi + lo with hi = v truncated to bf16 (its top 16 bits, a byte permute)
@@ -180,9 +190,14 @@ __device__ __forceinline__ void split2(uint64_t v, uint32_t &hi, uint32_t &lo) {
 }
 
 // round_half_even(y * inv) as an int, valid for |y * inv| < 2^22 (alpha >= 2^-19):
-// adding 1.5 * 2^23 leaves the rounded integer in the low mantissa bits.
-__device__ __forceinline__ int round_code(uint32_t ybits, float inv) {
-    return __float_as_int(fmaf(__uint_as_float(ybits), inv, 12582912.0f)) - 0x4B400000;
+// adding 1.5 * 2^23 leaves the rounded integer in the low mantissa bits.  The
+// offset is removed by an integer multiply-add with `one` (== 1, loaded at run
+// time), which runs beside the floating-point work instead of on the logic pipe.
+__device__ __forceinline__ int round_code(uint32_t ybits, float inv, int one) {
+    const int b = __float_as_int(fmaf(__uint_as_float(ybits), inv, 12582912.0f));
+    int k;
+    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k) : "r"(b), "r"(one), "r"(-0x4B400000));
+    return k;
 }
 
 // Position in a ring of n barrier-guarded slots: slot index and the parity of
@@ -239,6 +254,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         mbar_init(bar(C::TEARDOWN), 1);
         *s_abort = 0;
+        *reinterpret_cast<int *>(smem + C::OFF_MISC + 8) = 1;  // `one` of round_code
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_x);
@@ -415,17 +431,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int t = warp < 8 ? tid - 64 : tid - 640 + 192;  // 0 .. kXThreads - 1
             constexpr int UPT = 16 * N1 / kXThreads;             // units per thread per group
             // thread t handles unit e = t + kXThreads u (u < UPT) of every group of the
-            // batch; its cinv values depend only on (u, t)
-            uint64_t cv[UPT][4];
+            // batch; its cinv values depend only on (u, t).  cinv = ch + cl, two bf16
+            // values (RN(cinv) and RN of the rest), so that x' needs only packed bf16
+            // arithmetic: hi = RN(x ch), lo = RN(x cl + RN(x ch - hi)).  Each step is one
+            // fused rounding; hi + lo is x * cinv to about 2^-14 relative.
+            uint32_t ch[UPT][4], cl[UPT][4];
 #pragma unroll
             for (int u = 0; u < UPT; ++u) {
                 const int e = t + kXThreads * u;
                 const int c = e / (8 * N1), rem = e % (8 * N1), r = rem >> 3, up = rem & 7;
                 const int b0 = (N2 == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
 #pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    cv[u][p] = uint64_t(__float_as_uint(cinv[r * N2 + b0 + 2 * p])) |
-                               (uint64_t(__float_as_uint(cinv[r * N2 + b0 + 2 * p + 1])) << 32);
+                for (int p = 0; p < 4; ++p) {
+                    const float c0 = cinv[r * N2 + b0 + 2 * p], c1 = cinv[r * N2 + b0 + 2 * p + 1];
+                    ch[u][p] = pack_bf16x2(c0, c1);
+                    cl[u][p] = pack_bf16x2(c0 - __uint_as_float(ch[u][p] << 16),
+                                           c1 - __uint_as_float(ch[u][p] & 0xFFFF0000u));
+                }
             }
             Ring rx, rc;
             for (int64_t j = 0; j < nb; ++j, rx.next(C::SX), rc.next(C::SC)) {
@@ -447,8 +469,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         uint32_t oh[4], ol[4];
 #pragma unroll
                         for (int p = 0; p < 4; ++p) {
-                            const uint64_t xv = uint64_t(w[p] << 16) | (uint64_t(w[p] & 0xFFFF0000u) << 32);
-                            split2(f32x2_mul(xv, cv[u][p]), oh[p], ol[p]);
+                            oh[p] = bf16x2_mul(w[p], ch[u][p]);
+                            const uint32_t rest = bf16x2_fma(w[p], ch[u][p], bf16x2_neg(oh[p]));
+                            ol[p] = bf16x2_fma(w[p], cl[u][p], rest);
                         }
                         *reinterpret_cast<uint4 *>(raw + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
                         *reinterpret_cast<uint4 *>(lo + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
@@ -496,10 +519,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp >= 12 && warp < 20) {
         // ---------------- epilogue: absmax, quantise, pack, store ----------------
-        // Two epilogue warpgroups take alternate groups.  Each thread reads two
-        // TMEM lanes (16x256b): lane g8 (even output column) and lane g8 + 8
-        // (odd column) of its 16-lane half, so both nibbles of every byte it
-        // writes are in its registers.
+        // Two epilogue warpgroups take alternate groups.  Each thread reads, with
+        // 16x256b loads, lanes g8 and g8 + 8 of both 16-lane halves of its warp's
+        // 32 lanes: four consecutive output columns (see lane_column), i.e. two
+        // whole bytes of each output row it covers, stored as one 16-bit word.
         const int ew = (warp - 12) >> 2;  // which epilogue warpgroup
         const int q = warp & 3;
         const int et = tid - 384 - 128 * ew;
@@ -507,8 +530,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int tok_h = (32 * q) / N2;
         const int g8 = lane >> 2, qq = lane & 3;
         float *red = s_red + 8 * ew;
+        const int one = *reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
         constexpr int NK = N1 / 16;
-        constexpr bool ONE_PASS = false;  // re-read TMEM: a group does not fit in 80 registers
         constexpr int V16_ROW = N2 / 32;     // 16-byte chunks per output row
         constexpr int V16 = C::H * N1 * V16_ROW;
         const uint32_t ng = uint32_t(nb) * C::GB;
@@ -541,30 +564,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (named_barrier_any(nbar, 128, !warp_ok)) break;
             __syncwarp();
             tc_fence_after();
-            uint32_t r[ONE_PASS ? 2 : 1][NK][8];
+            // absmax from a first read (32x32b, thread = lane), 32 columns per load
             float mx4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            if (ONE_PASS) {
-#pragma unroll
-                for (int hf = 0; hf < (ONE_PASS ? 2 : 1); ++hf) {
-                    const uint32_t taddr = tmem + (uint32_t(32 * q + 16 * hf) << 16) + C::R2(int(b));
-                    if (N1 == 64)
-                        tmem_ld_16x256b_x8(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[hf][0][0]));
-                    else
-#pragma unroll
-                        for (int cc = 0; cc < NK; ++cc) tmem_ld_16x256b_x2(taddr + 16 * cc, r[hf][cc]);
-                }
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(bar(C::D2EMPTY + b));  // D2 region free for the next stage 2
-#pragma unroll
-                for (int hf = 0; hf < (ONE_PASS ? 2 : 1); ++hf)
-#pragma unroll
-                    for (int cc = 0; cc < NK; ++cc)
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            mx4[e & 3] = fmaxf(mx4[e & 3], fabsf(__uint_as_float(r[hf][cc][e])));
-            } else {
-                // absmax from a first read (32x32b, thread = lane), 32 columns per load
+            {
                 const uint32_t lane_off = uint32_t(32 * q) << 16;
                 if (N1 % 32 == 0) {
 #pragma unroll
@@ -573,7 +575,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         tmem_ld_32x32b_x32(tmem + lane_off + C::R2(int(b)) + k0, v);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], fabsf(__uint_as_float(v[e])));
+                        for (int e = 0; e < 32; e += 8) {
+                            mx4[0] = fmax3(mx4[0], fabsf(__uint_as_float(v[e])), fabsf(__uint_as_float(v[e + 1])));
+                            mx4[1] = fmax3(mx4[1], fabsf(__uint_as_float(v[e + 2])), fabsf(__uint_as_float(v[e + 3])));
+                            mx4[2] = fmax3(mx4[2], fabsf(__uint_as_float(v[e + 4])), fabsf(__uint_as_float(v[e + 5])));
+                            mx4[3] = fmax3(mx4[3], fabsf(__uint_as_float(v[e + 6])), fabsf(__uint_as_float(v[e + 7])));
+                        }
                     }
                 } else {
 #pragma unroll
@@ -582,11 +589,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         tmem_ld_32x32b_x16(tmem + lane_off + C::R2(int(b)) + 16 * k0, v);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], fabsf(__uint_as_float(v[e])));
+                        for (int e = 0; e < 16; e += 8) {
+                            mx4[0] = fmax3(mx4[0], fabsf(__uint_as_float(v[e])), fabsf(__uint_as_float(v[e + 1])));
+                            mx4[1] = fmax3(mx4[1], fabsf(__uint_as_float(v[e + 2])), fabsf(__uint_as_float(v[e + 3])));
+                            mx4[2] = fmax3(mx4[2], fabsf(__uint_as_float(v[e + 4])), fabsf(__uint_as_float(v[e + 5])));
+                            mx4[3] = fmax3(mx4[3], fabsf(__uint_as_float(v[e + 6])), fabsf(__uint_as_float(v[e + 7])));
+                        }
                     }
                 }
             }
-            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            const float mx = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
             // non-negative floats order like their bit patterns: one warp reduction
             const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
             if (lane == 0) red[4 * buf + q] = __uint_as_float(wmax);
@@ -602,37 +614,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const float s = alpha * m * (1.0f / 7.0f);
             const float inv = s > 0.0f ? fminf(__fdividef(1.0f, s), 3.0e38f) : 0.0f;
             unsigned char *stg = smem + C::OFF_STG + (2 * ew + buf) * C::STG;
+            // this thread's two bytes of every row: columns 4 g8 .. 4 g8 + 3 of the warp's 32
+            unsigned char *rowbase = stg + (tok_h * N1) * C::RS + ((32 * q) % N2) / 2 + 2 * g8;
+            const uint32_t t0 = tmem + (uint32_t(32 * q) << 16) + C::R2(int(b));
+            constexpr int CB = N1 % 32 == 0 ? 2 : 1;  // 16-column chunks per load
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int L0 = 32 * q + 16 * hf;
-                const int col_byte = 8 * ((L0 % N2) / 16) + g8;
-                unsigned char *rowbase = stg + (tok_h * N1) * C::RS + col_byte;
-                uint32_t rl[NK][8];
-                if (!ONE_PASS) {
-                    if (N1 == 64)
-                        tmem_ld_16x256b_x8(tmem + (uint32_t(L0) << 16) + C::R2(int(b)),
-                                           *reinterpret_cast<uint32_t(*)[32]>(&rl[0][0]));
-                    else
-#pragma unroll
-                        for (int cc = 0; cc < NK; ++cc)
-                            tmem_ld_16x256b_x2(tmem + (uint32_t(L0) << 16) + C::R2(int(b)) + 16 * cc, rl[cc]);
-                    tmem_wait_ld();
-                    if (hf == 1) {
-                        tc_fence_before();
-                        mbar_arrive(bar(C::D2EMPTY + b));
-                    }
+            for (int c0 = 0; c0 < NK; c0 += CB) {
+                // half 0 (lanes 32 q + [0, 16)) and half 1 (lanes 32 q + [16, 32))
+                uint32_t ra[8 * CB], rb[8 * CB];
+                if (CB == 2) {
+                    tmem_ld_16x256b_x4(t0 + 16 * c0, *reinterpret_cast<uint32_t(*)[16]>(ra));
+                    tmem_ld_16x256b_x4(t0 + (16u << 16) + 16 * c0, *reinterpret_cast<uint32_t(*)[16]>(rb));
+                } else {
+                    tmem_ld_16x256b_x2(t0 + 16 * c0, *reinterpret_cast<uint32_t(*)[8]>(ra));
+                    tmem_ld_16x256b_x2(t0 + (16u << 16) + 16 * c0, *reinterpret_cast<uint32_t(*)[8]>(rb));
+                }
+                tmem_wait_ld();
+                if (c0 + CB >= NK) {
+                    tc_fence_before();
+                    mbar_arrive(bar(C::D2EMPTY + b));  // D2 region free for the next stage 2
                 }
 #pragma unroll
-                for (int cc = 0; cc < NK; ++cc) {
+                for (int rep = 0; rep < 2 * CB; ++rep) {
+                    const int i0 = 16 * c0 + 8 * rep + 2 * qq;
 #pragma unroll
-                    for (int rep = 0; rep < 2; ++rep) {
-                        const int i0 = 16 * cc + 8 * rep + 2 * qq;
-                        const uint32_t *rr = ONE_PASS ? &r[hf & (ONE_PASS ? 1 : 0)][cc][4 * rep] : &rl[cc][4 * rep];
-                        // byte(i0) = even | odd << 4, byte(i0 + 1) likewise; saturate to [-8, 7]
-                        const uint32_t w0 = pack_s4x2(round_code(rr[2], inv), round_code(rr[0], inv), 0u);
-                        const uint32_t w1 = pack_s4x2(round_code(rr[3], inv), round_code(rr[1], inv), w0);
-                        rowbase[i0 * C::RS] = uint8_t(w1 >> 8);
-                        rowbase[(i0 + 1) * C::RS] = uint8_t(w1);
+                    for (int d = 0; d < 2; ++d) {
+                        // row i0 + d: columns 4 g8 + (0, 1) from half 0, + (2, 3) from half 1;
+                        // byte = even column in the low nibble, odd in the high one
+                        const uint32_t wb = pack_s4x2(round_code(rb[4 * rep + 2 + d], inv, one),
+                                                      round_code(rb[4 * rep + d], inv, one), 0u);
+                        const uint32_t w = pack_s4x2(round_code(ra[4 * rep + 2 + d], inv, one),
+                                                     round_code(ra[4 * rep + d], inv, one), wb);
+                        *reinterpret_cast<uint16_t *>(rowbase + (i0 + d) * C::RS) = uint16_t(w);
                     }
                 }
             }
