@@ -7,9 +7,9 @@
 // then per-token absmax, s = alpha * max / 7, round-half-even codes clamped
 // to [-8, 7], packed two per byte.  Only codes and scales reach HBM.
 //
-// Layout of the work (one CTA per SM, 22 warps, groups of H = 128 / n2
+// Layout of the work (one CTA per SM, 24 warps, groups of H = 128 / n2
 // tokens so that the 128 TMEM lanes always hold 128 output columns; stage 1
-// runs on batches of GB groups so that its MMAs are 128 wide):
+// runs on batches of GB groups, MMAs up to 128 columns wide):
 //   TMEM lane l = (h, m): token h of the group, output column
 //   j = lane_column(m) of its n2 columns.  Within each block of 32 lanes the
 //   columns are interleaved so that the thread of a 16x256b TMEM load that
@@ -22,17 +22,16 @@
 //   convert (TMEM)    D1 fp32 -> A2 = hi + lo bf16, in place, chunk by chunk.
 //   stage 2 (TS MMA)  D2[l][i]  = sum_a A2[l][a] * P1[a][i]   (A from TMEM)
 //   epilogue          absmax over the token's lanes, quantise, pack into a
-//                     bank-spread staging area, 16-byte stores to HBM.
+//                     swizzled staging tile, one TMA store per group to HBM.
 // With cinv, the x' split warps turn each raw x tile into x' = x * cinv
 // split into a hi bf16 tile (written over x) and a lo bf16 tile; stage 1
 // then accumulates both.  TMEM holds P2^T, two D1/A2 regions (batches) and
-// three D2 regions (groups, n1 <= 64), so that stage 2 of batch k - 1 is
-// issued after stage 1 of batch k and the tensor pipe never waits for work
-// the issuer has just queued.
+// three D2 regions (groups, n1 <= 64).
 //
-// Warp roles: 0 TMA producer | 1 TMEM allocator + MMA issuer | 2-7, 20-21 x'
-// split (cinv only) | 8-11 P2^T into TMEM, then D1 -> A2 conversion | 12-15
-// and 16-19 two epilogue warpgroups taking alternate groups.  Every mbarrier
+// Warp roles: 0 TMA producer | 1 TMEM allocator + stage-1 MMA issuer | 5
+// stage-2 MMA issuer | 2-4, 6-7, 20, 22-23 x' split (cinv only) | 8-11 P2^T
+// into TMEM, then D1 -> A2 conversion | 12-15 and 16-19 two epilogue
+// warpgroups taking alternate groups | 21 idle.  Every mbarrier
 // wait is bounded: after about a second it ORs a site bit into
 // g_device_error, raises a CTA-wide abort flag and the roles drain and exit.
 #include <cuda.h>
@@ -64,8 +63,26 @@ namespace {
 
 using namespace tc;
 
-constexpr int kTcThreads = 704;  // 22 warps, at most 88 registers per thread
-constexpr int kXThreads = 256;   // x' split: warps 2-7 and 20-21
+constexpr int kTcThreads = 768;  // 24 warps, at most 80 registers per thread
+constexpr int kXThreads = 256;   // x' split: warps 2-4, 6-7, 20, 22-23
+
+// Warp w runs on scheduler w % 4.  The x' split warps avoid scheduler 1, which
+// runs the MMA issuers: their instruction streams are short but on the
+// critical path.
+// Returns the x' split warp's index in [0, 8), or -1.
+__device__ __forceinline__ int xsplit_index(int warp) {
+    switch (warp) {
+    case 2: return 0;
+    case 3: return 1;
+    case 4: return 2;
+    case 6: return 3;
+    case 7: return 4;
+    case 20: return 5;
+    case 22: return 6;
+    case 23: return 7;
+    default: return -1;
+    }
+}
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // about one second
 
 enum : unsigned {
@@ -110,10 +127,10 @@ __host__ __device__ constexpr int imax(int a, int b) { return a > b ? a : b; }
 template <int N1, int N2, bool SCALED>
 struct Cfg {
     static constexpr int H = 128 / N2;               // tokens stacked in the TMEM lanes
-    static constexpr int N = N1 * N2;
-    // Stage 1 runs on batches of GB groups so that its MMAs are N = GB * n1 wide.
-    static constexpr int GB = N1 <= 64 ? 128 / N1 > 8 ? 8 : 128 / N1 : 1;
-    static constexpr int NS1 = GB * N1;              // stage-1 MMA N (<= 128)
+    // Stage 1 runs on batches of GB groups so that its MMAs are N = GB * n1 wide
+    // (up to 128).
+    static constexpr int GB = N1 <= 64 ? imin(8, 128 / N1) : 1;
+    static constexpr int NS1 = GB * N1;              // stage-1 MMA N
     static constexpr int CHUNK = NS1 * 128;          // one 64-element K chunk of a batch tile
     static constexpr int XTILE = 2 * CHUNK;          // a batch's x tile (K = 128)
     static constexpr int NCH2 = (N1 + 63) / 64;      // K chunks of P1^T
@@ -122,22 +139,22 @@ struct Cfg {
     // P2^T lives in TMEM (stage 1 reads A from TMEM) when the columns allow it.
     static constexpr bool A1_TMEM = N1P <= 96;
     static constexpr int A1COLS = A1_TMEM ? 64 : 0;  // 128 K-elements of bf16
-    static constexpr int NB1 = 2;                    // D1/A2 regions (batches)
-    static constexpr int NB2 = (A1COLS + NB1 * R1W + 3 * N1P <= 512) ? 3 : 2;  // D2 regions (groups)
+    static constexpr int NB2 = (A1COLS + 2 * R1W + 3 * N1P <= 512) ? 3 : 2;       // D2 regions (groups)
+    static constexpr int NB1 = imin(4, (512 - A1COLS - NB2 * N1P) / R1W);        // D1/A2 regions (batches)
     static constexpr int TMEM_USED = A1COLS + NB1 * R1W + NB2 * N1P;
     static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
-    static constexpr int SC = 2;                     // lo-half tile stages (cinv); hi is written in place
-    static constexpr int RS = N2 / 2 + 16;           // staging row stride (bytes), bank-spread
-    static constexpr int STG = H * N1 * RS;          // staging bytes per group
+    static constexpr int RB = N2 / 2;                // bytes of one output row (codes)
+    static constexpr int STG = H * N1 * RB;          // staging bytes per group (a multiple of 1024)
     static constexpr int OFF_B2 = 0;
     static constexpr int OFF_A1 = align_up(OFF_B2 + NCH2 * N1 * 128, 1024);
-    static constexpr int OFF_RAW = OFF_A1 + (A1_TMEM ? 0 : 32768);
-    static constexpr int FIXED = OFF_RAW + (SCALED ? SC * XTILE : 0) + 4 * STG + 2048;
-    static constexpr int SX = imax(2, imin(8, (222 * 1024 - FIXED) / XTILE));  // raw x stages
+    static constexpr int OFF_STG = OFF_A1 + (A1_TMEM ? 0 : 32768);  // 2 epilogues x 2 staging buffers
+    static constexpr int OFF_RAW = OFF_STG + 4 * STG;
+    static constexpr int BUDGET = 222 * 1024 - OFF_RAW - 2048;
+    static constexpr int SC = (SCALED && BUDGET >= 10 * XTILE) ? 4 : 2;  // lo-half tile stages (cinv)
+    static constexpr int SX = imax(2, imin(8, (BUDGET - (SCALED ? SC * XTILE : 0)) / XTILE));  // raw x stages
     static constexpr int OFF_CONV = OFF_RAW + SX * XTILE;
-    static constexpr int OFF_STG = OFF_CONV + (SCALED ? SC * XTILE : 0);
     static constexpr int NBAR = 2 * SX + 2 * SC + 3 * NB1 + 2 * NB2 + 1;
-    static constexpr int OFF_BAR = align_up(OFF_STG + 4 * STG, 16);  // 2 epilogues x 2 staging buffers
+    static constexpr int OFF_BAR = align_up(OFF_CONV + (SCALED ? SC * XTILE : 0), 16);
     static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem base, abort flag, the constant 1, 2 x 2 x 4 maxima
     static constexpr int SMEM = OFF_MISC + 80 + 1024;    // + slack for 1024-byte alignment
     // barrier indices
@@ -148,11 +165,23 @@ struct Cfg {
     static_assert(N1 % 16 == 0 && N1 >= 16 && N1 <= 128, "n1 must be a multiple of 16 in [16, 128]");
     static_assert(!SCALED || N1 <= 64, "x' split keeps cinv in registers: n1 <= 64");
     static_assert(NS1 % 16 == 0 && NS1 <= 128, "stage-1 MMA width");
+    static_assert(NB1 >= 2, "stage-1 regions");
     static_assert(TMEM_USED <= 512, "TMEM budget");
+    static_assert(STG % 1024 == 0 && OFF_STG % 1024 == 0 && OFF_RAW % 1024 == 0, "swizzle alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
     __host__ __device__ static constexpr uint32_t R1(int b) { return uint32_t(A1COLS + b * R1W); }
     __host__ __device__ static constexpr uint32_t R2(int b) { return uint32_t(A1COLS + NB1 * R1W + b * N1P); }
 };
+
+// Offset of byte b of staging row r: rows of n2/2 bytes with the 16-byte chunks
+// permuted the way a TMA store with 64-byte (n2 = 128) or 32-byte (n2 = 64)
+// swizzle reads them back in order.  It also spreads the epilogue's 16-bit
+// stores over all banks.
+template <int N2>
+__device__ __forceinline__ uint32_t stg_offset(int r, int b) {
+    const int swz = N2 == 128 ? (r >> 1) & 3 : (r >> 2) & 1;
+    return uint32_t(r * (N2 / 2) + ((((b >> 4) ^ swz) << 4) | (b & 15)));
+}
 
 // Byte offset of element (row r, k in [0, 64)) inside one 128B-swizzled chunk.
 __device__ __forceinline__ uint32_t swz128(int r, int k) {
@@ -214,9 +243,10 @@ struct Ring {
 
 template <int N1, int N2, bool SCALED>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    kq_tc05_fused_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t *__restrict__ P1,
+    kq_tc05_fused_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
+                         const uint16_t *__restrict__ P1,
                          const uint16_t *__restrict__ P2, const float *__restrict__ cinv, float alpha,
-                         uint8_t *__restrict__ q_out, float *__restrict__ scale_out, int64_t T) {
+                         float *__restrict__ scale_out, int64_t T) {
     using C = Cfg<N1, N2, SCALED>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -252,12 +282,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(bar(C::D2FULL + b), 1);
             mbar_init(bar(C::D2EMPTY + b), 128);
         }
-        mbar_init(bar(C::TEARDOWN), 1);
+        mbar_init(bar(C::TEARDOWN), 2);  // one commit from each MMA issuer
         *s_abort = 0;
         *reinterpret_cast<int *>(smem + C::OFF_MISC + 8) = 1;  // `one` of round_code
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_x);
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmap_x);
+        prefetch_tensormap(&tmap_q);
+    }
     if (warp == 1) {
         tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
         tmem_relinquish();
@@ -300,10 +333,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // Release of x tiles: stage 1 of a batch finishing (seen by the D1 -> A2
-    // converters) frees its tile; the last stage 2 of a batch finishing (seen
-    // by the epilogue) frees its D1/A2 region.  The MMA thread only commits
-    // D1FULL (once per batch) and D2FULL (once per group).
+    // Buffer hand-offs from the tensor pipe are commits by the MMA warp: stage 1
+    // of a batch completing frees its x (and lo) tile and fills its D1 region;
+    // stage 2 of a group completing fills a D2 region; stage 2 of a whole batch
+    // completing frees its D1/A2 region.
     if (warp == 0) {
         // ---------------- TMA producer: one batch tile per slot ----------------
         // The whole warp runs the loop (converged); one elected lane issues.
@@ -339,20 +372,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (i + C::SX >= issued)
                 wait_bounded(bar(C::FULL + rd.idx), rd.phase, s_abort, kSiteDrain, kWaitLimitNs, true);
         __syncwarp();
-    } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        // The whole warp runs the loop and the waits (converged, so every
-        // operand is warp-uniform); one elected lane issues MMAs and commits.
+    } else if (warp == 1 || warp == 5) {
+        // ---------------- MMA issuers: warp 1 stage 1, warp 5 stage 2 ----------------
+        // Each runs its loop and waits converged (every operand warp-uniform); one
+        // elected lane issues the MMAs and commits.  Two issuers keep the latency of
+        // one stage's waits and commits off the other's critical path; each commit
+        // covers the MMAs its own thread issued.
         constexpr uint32_t idesc1 = idesc_bf16_f32(128, C::NS1);
         constexpr uint32_t idesc2 = idesc_bf16_f32(128, N1);
-        const uint64_t b2d = sdesc_kmajor_sw128(sbase + C::OFF_B2);
+        const uint32_t b2l = sdesc_sw128_lo(sbase + C::OFF_B2);
         const uint64_t a1d = sdesc_kmajor_sw128(sbase + C::OFF_A1);
         // descriptor start addresses are in 16-byte units in the low bits
-        auto koff1 = [](int kk) { return uint64_t(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4); };
-        auto koff2 = [](int kk) { return uint64_t(((kk >> 2) * (N1 * 128) + (kk & 3) * 32) >> 4); };
-        Ring rin, rxs, r1, r1p, r2;  // input tiles, raw slots, D1/A2 regions (stage 1 / 2), D2 regions
-        for (int64_t j = 0; j <= nb; ++j) {
-            if (j < nb) {  // stage 1 of batch j
+        auto koff1 = [](int kk) { return uint32_t(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4); };
+        auto koff2 = [](int kk) { return uint32_t(((kk >> 2) * (N1 * 128) + (kk & 3) * 32) >> 4); };
+        if (warp == 1) {
+            Ring rin, rxs, r1;  // input tiles, raw slots, D1/A2 regions
+            for (int64_t j = 0; j < nb; ++j) {
                 bool ok = wait_bounded(bar(C::D1EMPTY + r1.idx), r1.phase ^ 1u, s_abort, kSiteMma, kWaitLimitNs,
                                        false);
                 uint32_t src, src_lo;
@@ -369,18 +404,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
                 const uint32_t d1 = tmem + C::R1(int(r1.idx));
-                const uint64_t bd_hi = sdesc_kmajor_sw128(src), bd_lo = sdesc_kmajor_sw128(src_lo);
+                const uint32_t bl_hi = sdesc_sw128_lo(src), bl_lo = sdesc_sw128_lo(src_lo);
                 if (elect_one()) {
 #pragma unroll
                     for (int pass = 0; pass < (SCALED ? 2 : 1); ++pass) {
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t b = (pass ? bd_lo : bd_hi) + koff1(kk);
-                            if (C::A1_TMEM)
-                                mma_ts(d1, tmem + 8 * kk, b, idesc1, (pass | kk) != 0);
-                            else
-                                mma_ss(d1, a1d + uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), b, idesc1,
-                                       (pass | kk) != 0);
+                            const uint32_t b = (pass ? bl_lo : bl_hi) + koff1(kk);
+                            if (C::A1_TMEM) {
+                                if ((pass | kk) != 0)
+                                    mma_ts_split<1>(d1, tmem + 8 * kk, b, kSdescSw128Hi, idesc1);
+                                else
+                                    mma_ts_split<0>(d1, tmem + 8 * kk, b, kSdescSw128Hi, idesc1);
+                            } else {
+                                const uint64_t a = a1d + uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                                if ((pass | kk) != 0)
+                                    mma_ss_split<1>(d1, a, b, kSdescSw128Hi, idesc1);
+                                else
+                                    mma_ss_split<0>(d1, a, b, kSdescSw128Hi, idesc1);
+                            }
                         }
                     }
                     tc_commit(bar(C::EMPTY + rxs.idx));  // x (hi) tile slot free
@@ -392,7 +434,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 rxs.next(C::SX);
                 r1.next(C::NB1);
             }
-            if (j >= 1) {  // stage 2 of every group of batch j - 1
+        } else {
+            Ring r1p, r2;  // D1/A2 regions, D2 regions
+            for (int64_t j = 0; j < nb; ++j) {
                 bool ok = wait_bounded(bar(C::A2FULL + r1p.idx), r1p.phase, s_abort, kSiteMma, kWaitLimitNs, false);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 const uint32_t a2b = tmem + C::R1(int(r1p.idx));
@@ -407,8 +451,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                         for (int pass = 0; pass < 2; ++pass)
 #pragma unroll
-                            for (int kk = 0; kk < N1 / 16; ++kk)
-                                mma_ts(d2, a2 + 16 * kk + 8 * pass, b2d + koff2(kk), idesc2, (pass | kk) != 0);
+                            for (int kk = 0; kk < N1 / 16; ++kk) {
+                                if ((pass | kk) != 0)
+                                    mma_ts_split<1>(d2, a2 + 16 * kk + 8 * pass, b2l + koff2(kk), kSdescSw128Hi,
+                                                    idesc2);
+                                else
+                                    mma_ts_split<0>(d2, a2 + 16 * kk + 8 * pass, b2l + koff2(kk), kSdescSw128Hi,
+                                                    idesc2);
+                            }
                         tc_commit(bar(C::D2FULL + r2.idx));
                     }
                     __syncwarp();
@@ -420,15 +470,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 r1p.next(C::NB1);
             }
         }
-        // Every MMA this warp issued has completed before TMEM is freed.
+        // Every MMA either issuer issued has completed before TMEM is freed.
         if (elect_one()) tc_commit(bar(C::TEARDOWN));
         __syncwarp();
         wait_bounded(bar(C::TEARDOWN), 0u, s_abort, kSiteDrain, kWaitLimitNs, true);
         __syncwarp();
-    } else if ((warp >= 2 && warp < 8) || warp >= 20) {
+    } else if (xsplit_index(warp) >= 0) {
         // ---------------- x' = x * cinv -> hi / lo bf16 tiles ----------------
         if (SCALED) {
-            const int t = warp < 8 ? tid - 64 : tid - 640 + 192;  // 0 .. kXThreads - 1
+            const int t = 32 * xsplit_index(warp) + lane;  // 0 .. kXThreads - 1
             constexpr int UPT = 16 * N1 / kXThreads;             // units per thread per group
             // thread t handles unit e = t + kXThreads u (u < UPT) of every group of the
             // batch; its cinv values depend only on (u, t).  cinv = ch + cl, two bf16
@@ -532,23 +582,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float *red = s_red + 8 * ew;
         const int one = *reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
         constexpr int NK = N1 / 16;
-        constexpr int V16_ROW = N2 / 32;     // 16-byte chunks per output row
-        constexpr int V16 = C::H * N1 * V16_ROW;
         const uint32_t ng = uint32_t(nb) * C::GB;
-        auto copy_out = [&](int64_t gprev, int sb) {
-            const int64_t tok0 = C::H * gprev;
-            const int64_t valid = (T - tok0) < C::H ? (T - tok0) : C::H;
-            const unsigned char *st = smem + C::OFF_STG + sb * C::STG;
-            uint8_t *gout = q_out + tok0 * (C::N / 2);
-#pragma unroll
-            for (int e0 = 0; e0 < V16; e0 += 128) {
-                const int e = e0 + et;
-                if (e < V16) {
-                    const int row = e / V16_ROW, c16 = e % V16_ROW;
-                    if (row < valid * N1)
-                        *reinterpret_cast<uint4 *>(gout + row * (N2 / 2) + 16 * c16) =
-                            *reinterpret_cast<const uint4 *>(st + row * C::RS + 16 * c16);
-                }
+        const uint32_t stg0 = sbase + C::OFF_STG + 2 * ew * C::STG;
+        // One thread per warpgroup writes a finished staging tile to HBM with a
+        // TMA store; the tensor map clips rows past the last token.
+        const bool storer = et == 0;
+        auto store_group = [&](int64_t gprev, int sb) {
+            if (storer) {
+                tma_store_2d(&tmap_q, 0, int(C::H * gprev * N1), stg0 + uint32_t(sb) * C::STG);
+                bulk_commit();
             }
         };
         int64_t g_prev = -1;
@@ -602,9 +644,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // non-negative floats order like their bit patterns: one warp reduction
             const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
             if (lane == 0) red[4 * buf + q] = __uint_as_float(wmax);
+            // the store that read this group's staging buffer (two groups back) is done
+            if (storer) bulk_wait_read<0>();
             // maxima visible; every thread finished writing its previous group's staging rows
             named_barrier_sync(nbar, 128);
-            if (g_prev >= 0) copy_out(g_prev, 2 * ew + (buf ^ 1));
+            if (g_prev >= 0) store_group(g_prev, buf ^ 1);
             float m = 0.0f;
 #pragma unroll
             for (int w = 0; w < 4; ++w)
@@ -615,7 +659,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const float inv = s > 0.0f ? fminf(__fdividef(1.0f, s), 3.0e38f) : 0.0f;
             unsigned char *stg = smem + C::OFF_STG + (2 * ew + buf) * C::STG;
             // this thread's two bytes of every row: columns 4 g8 .. 4 g8 + 3 of the warp's 32
-            unsigned char *rowbase = stg + (tok_h * N1) * C::RS + ((32 * q) % N2) / 2 + 2 * g8;
+            const int row0 = tok_h * N1, bcol = ((32 * q) % N2) / 2 + 2 * g8;
             const uint32_t t0 = tmem + (uint32_t(32 * q) << 16) + C::R2(int(b));
             constexpr int CB = N1 % 32 == 0 ? 2 : 1;  // 16-column chunks per load
 #pragma unroll
@@ -645,17 +689,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                                       round_code(rb[4 * rep + d], inv, one), 0u);
                         const uint32_t w = pack_s4x2(round_code(ra[4 * rep + 2 + d], inv, one),
                                                      round_code(ra[4 * rep + d], inv, one), wb);
-                        *reinterpret_cast<uint16_t *>(rowbase + (i0 + d) * C::RS) = uint16_t(w);
+                        *reinterpret_cast<uint16_t *>(stg + stg_offset<N2>(row0 + i0 + d, bcol)) = uint16_t(w);
                     }
                 }
             }
+            fence_proxy_async_smem();  // staging writes visible to the TMA store
             const int64_t tok0 = C::H * g;
             if (lane == 0 && (32 * q) % N2 == 0 && tok0 + tok_h < T) scale_out[tok0 + tok_h] = s;
             g_prev = g;
         }
         // the last group's rows: everyone has written them once all pass this barrier
         named_barrier_sync(nbar, 128);
-        if (g_prev >= 0) copy_out(g_prev, 2 * ew + ((it - 1) & 1));
+        if (g_prev >= 0) store_group(g_prev, (it - 1) & 1);
+        if (storer) bulk_wait<0>();  // staging is read (and written out) before the CTA exits
     }
 
     tc_fence_before();
@@ -719,10 +765,19 @@ cudaError_t launch_inst(const LaunchArgs &a) {
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    // codes: rows of n2/2 bytes, one box = one group's H * n1 rows, swizzled like the staging tile
+    CUtensorMap tmap_q;
+    const cuuint64_t qdims[2] = {cuuint64_t(C::RB), cuuint64_t(a.T) * N1};
+    const cuuint64_t qstrides[1] = {cuuint64_t(C::RB)};
+    const cuuint32_t qbox[2] = {cuuint32_t(C::RB), cuuint32_t(C::H * N1)};
+    r = encode(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.q_out, qdims, qstrides, qbox, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, N2 == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     const int64_t G = (a.T + C::H - 1) / C::H;
     const int64_t NBt = (G + C::GB - 1) / C::GB;
     const int64_t grid = NBt < a.num_sms ? NBt : a.num_sms;
-    kern<<<unsigned(grid), kTcThreads, C::SMEM, a.stream>>>(tmap, a.P1, a.P2, a.cinv, a.alpha, a.q_out,
+    kern<<<unsigned(grid), kTcThreads, C::SMEM, a.stream>>>(tmap, tmap_q, a.P1, a.P2, a.cinv, a.alpha,
                                                             a.scale_out, a.T);
     return cudaGetLastError();
 }
