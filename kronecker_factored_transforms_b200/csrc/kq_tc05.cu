@@ -178,9 +178,33 @@ struct Cfg {
 // swizzle reads them back in order.  It also spreads the epilogue's 16-bit
 // stores over all banks.
 template <int N2>
-__device__ __forceinline__ uint32_t stg_offset(int r, int b) {
+__host__ __device__ constexpr uint32_t stg_offset(int r, int b) {
     const int swz = N2 == 128 ? (r >> 1) & 3 : (r >> 2) & 1;
     return uint32_t(r * (N2 / 2) + ((((b >> 4) ^ swz) << 4) | (b & 15)));
+}
+
+// The epilogue writes staging row row0 + 16 c + 8 rep + 2 qq + d, byte column
+// bcol, at base(qq, bcol) + (16 c + 8 rep + d) * n2/2; checked here against
+// stg_offset for every thread and store of an n1 x n2 group.
+template <int N1, int N2>
+__host__ __device__ constexpr bool staging_addresses_match() {
+    constexpr int H = 128 / N2, RB = N2 / 2;
+    for (int q = 0; q < 4; ++q)
+        for (int g8 = 0; g8 < 8; ++g8)
+            for (int qq = 0; qq < 4; ++qq) {
+                const int row0 = ((32 * q) / N2) * N1, bcol = ((32 * q) % N2) / 2 + 2 * g8;
+                const int swz_t = N2 == 128 ? qq : (qq >> 1);
+                const int base = (row0 + 2 * qq) * RB + ((((bcol >> 4) ^ swz_t) << 4) | (bcol & 15));
+                for (int c = 0; c < N1 / 16; ++c)
+                    for (int rep = 0; rep < 2; ++rep)
+                        for (int d = 0; d < 2; ++d) {
+                            const int r = row0 + 16 * c + 8 * rep + 2 * qq + d;
+                            if (r >= H * N1 || uint32_t(base + (16 * c + 8 * rep + d) * RB) != stg_offset<N2>(r, bcol) ||
+                                uint32_t(base + (16 * c + 8 * rep + d) * RB) + 2 > uint32_t(H * N1 * RB))
+                                return false;
+                        }
+            }
+    return true;
 }
 
 // Byte offset of element (row r, k in [0, 64)) inside one 128B-swizzled chunk.
@@ -195,6 +219,18 @@ __device__ __forceinline__ uint32_t swz128(int r, int k) {
 __host__ __device__ constexpr int lane_column(int m) {
     return (m & ~31) | ((m & 7) << 2) | (((m >> 4) & 1) << 1) | ((m >> 3) & 1);
 }
+
+// Inverse of lane_column: the lane (within a token) that holds output column j.
+__host__ __device__ constexpr int lane_of_column(int j) {
+    return (j & ~31) | (((j >> 1) & 1) << 4) | ((j & 1) << 3) | ((j >> 2) & 7);
+}
+
+__host__ __device__ constexpr bool lane_maps_invert() {
+    for (int m = 0; m < 128; ++m)
+        if (lane_of_column(lane_column(m)) != m || lane_column(m) >= 128) return false;
+    return true;
+}
+static_assert(lane_maps_invert(), "lane_of_column inverts lane_column");
 
 // Row l of A1 = block-diag over the stacked tokens of P2^T, rows permuted:
 // A1[l][k] = P2[b][lane_column(m)] for l = (h, m), k = (h, b); zero off the
@@ -218,14 +254,20 @@ __device__ __forceinline__ void split2(uint64_t v, uint32_t &hi, uint32_t &lo) {
     lo = pack_bf16x2(__uint_as_float(uint32_t(l)), __uint_as_float(uint32_t(l >> 32)));
 }
 
-// round_half_even(y * inv) as an int, valid for |y * inv| < 2^22 (alpha >= 2^-19):
-// adding 1.5 * 2^23 leaves the rounded integer in the low mantissa bits.  The
-// offset is removed by an integer multiply-add with `one` (== 1, loaded at run
-// time), which runs beside the floating-point work instead of on the logic pipe.
-__device__ __forceinline__ int round_code(uint32_t ybits, float inv, int one) {
-    const int b = __float_as_int(fmaf(__uint_as_float(ybits), inv, 12582912.0f));
+// round_half_even(y * inv) for two values at once, valid for |y * inv| < 2^22
+// (alpha >= 2^-19): adding 1.5 * 2^23 leaves the rounded integer in the low
+// mantissa bits of each fp32 result (bit patterns 0x4B400000 + k).
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;  // 1.5 * 2^23
+__device__ __forceinline__ uint64_t round_codes2(uint32_t y0, uint32_t y1, uint64_t inv2) {
+    constexpr uint64_t magic2 = uint64_t(kRoundMagicBits) | (uint64_t(kRoundMagicBits) << 32);
+    return f32x2_fma(uint64_t(y0) | (uint64_t(y1) << 32), inv2, magic2);
+}
+// The integer k of one such result.  The offset is removed by an integer
+// multiply-add with `one` (== 1, loaded at run time), which runs beside the
+// floating-point work instead of on the logic pipe.
+__device__ __forceinline__ int code_of(uint32_t bits, int one) {
     int k;
-    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k) : "r"(b), "r"(one), "r"(-0x4B400000));
+    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k) : "r"(bits), "r"(one), "r"(-int(kRoundMagicBits)));
     return k;
 }
 
@@ -248,6 +290,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                          const uint16_t *__restrict__ P2, const float *__restrict__ cinv, float alpha,
                          float *__restrict__ scale_out, int64_t T) {
     using C = Cfg<N1, N2, SCALED>;
+    static_assert(staging_addresses_match<N1, N2>(), "epilogue staging addresses");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
@@ -296,43 +339,101 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_relinquish();
     }
 
-    // B2[i][a] = P1[a][i] (rows i, K = a), 128B-swizzled K-major, zero beyond a = n1.
-    for (int e = tid; e < C::NCH2 * 64 * N1; e += kTcThreads) {
-        const int i = e / (C::NCH2 * 64), ka = e % (C::NCH2 * 64);
-        const uint16_t v = ka < N1 ? P1[ka * N1 + i] : uint16_t(0);
-        *reinterpret_cast<uint16_t *>(smem + C::OFF_B2 + (ka >> 6) * (N1 * 128) + swz128(i, ka & 63)) = v;
-    }
-    if (!C::A1_TMEM) {
-        for (int e = tid; e < 128 * 128; e += kTcThreads) {
-            const int l = e >> 7, k = e & 127;
-            *reinterpret_cast<uint16_t *>(smem + C::OFF_A1 + (k >> 6) * 16384 + swz128(l, k & 63)) =
-                a1_value<N2>(P2, l, k);
-        }
-    }
-    fence_proxy_async_smem();
+    // Barriers and the TMEM address are published.  The TMA producer and the x'
+    // split start at once; the other warps first build the factor operands, so
+    // that building them overlaps the first loads of x.
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    if (C::A1_TMEM && warp >= 8 && warp < 12) {
-        // A1 into TMEM columns [0, 64): lane l holds row l, K pairs packed per column.
-        const int l = 32 * (warp & 3) + lane;
-        const uint32_t taddr = tmem + (uint32_t(32 * (warp & 3)) << 16);
+    const int setup_idx = warp == 1 ? 0 : warp == 5 ? 1 : (warp >= 8 && warp < 20) ? warp - 6 : warp == 21 ? 14 : -1;
+    if (setup_idx >= 0) {
+        constexpr int kSetupThreads = 15 * 32;
+        const int st = 32 * setup_idx + lane;
+        // B2[i][a] = P1[a][i] (rows i, K = a), 128B-swizzled K-major, zero beyond a = n1.
+        // Each thread reads whole 16-byte pieces of rows of P1 (all its loads first)
+        // and scatters their eight values down a column of B2.
+        {
+            constexpr int PIECES = N1 * N1 / 8, PER = (PIECES + kSetupThreads - 1) / kSetupThreads;
+            uint4 v[PER];
 #pragma unroll
-        for (int kc = 0; kc < 4; ++kc) {
-            uint32_t w[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int k = 32 * kc + 2 * e;
-                w[e] = uint32_t(a1_value<N2>(P2, l, k)) | (uint32_t(a1_value<N2>(P2, l, k + 1)) << 16);
+            for (int u = 0; u < PER; ++u) {
+                const int c = st + u * kSetupThreads;
+                if (c < PIECES) v[u] = *reinterpret_cast<const uint4 *>(P1 + 8 * c);
             }
-            tmem_st_32x32b_x16(taddr + 16 * kc, w);
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int c = st + u * kSetupThreads;
+                if (c < PIECES) {
+                    const int a = (8 * c) / N1, i0 = (8 * c) % N1;
+                    const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                    for (int t = 0; t < 8; ++t)
+                        *reinterpret_cast<uint16_t *>(smem + C::OFF_B2 + (a >> 6) * (N1 * 128) + swz128(i0 + t, a & 63)) =
+                            uint16_t(w[t >> 1] >> (16 * (t & 1)));
+                }
+            }
+            // zero K padding (a in [n1, 64 NCH2))
+            for (int e = st; e < (C::NCH2 * 64 - N1) * N1; e += kSetupThreads) {
+                const int a = N1 + e / N1, i = e % N1;
+                *reinterpret_cast<uint16_t *>(smem + C::OFF_B2 + (a >> 6) * (N1 * 128) + swz128(i, a & 63)) = 0;
+            }
         }
-        tmem_wait_st();
+        if (!C::A1_TMEM) {
+            // A1[(h, m)][(h', b)] = P2[b][lane_column(m)] if h == h' else 0, from
+            // 16-byte pieces of rows of P2 (loads first), 128B-swizzled K-major.
+            constexpr int PIECES = N2 * N2 / 8, PER = (PIECES + kSetupThreads - 1) / kSetupThreads;
+            uint4 v[PER];
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int c = st + u * kSetupThreads;
+                if (c < PIECES) v[u] = *reinterpret_cast<const uint4 *>(P2 + 8 * c);
+            }
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int c = st + u * kSetupThreads;
+                if (c < PIECES) {
+                    const int b = (8 * c) / N2, j0 = (8 * c) % N2;
+                    const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        const int m = lane_of_column(j0 + t);
+#pragma unroll
+                        for (int h = 0; h < C::H; ++h)
+#pragma unroll
+                            for (int hk = 0; hk < C::H; ++hk) {
+                                const int l = h * N2 + m, k = hk * N2 + b;
+                                *reinterpret_cast<uint16_t *>(smem + C::OFF_A1 + (k >> 6) * 16384 + swz128(l, k & 63)) =
+                                    h == hk ? uint16_t(w[t >> 1] >> (16 * (t & 1))) : uint16_t(0);
+                            }
+                    }
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        if (C::A1_TMEM && warp >= 8 && warp < 16) {
+            // A1 into TMEM columns [0, 64): lane l holds row l, K pairs packed per
+            // column; warps 8-11 write K in [0, 64), warps 12-15 K in [64, 128).
+            const int l = 32 * (warp & 3) + lane;
+            const uint32_t taddr = tmem + (uint32_t(32 * (warp & 3)) << 16);
+            const int kc0 = warp < 12 ? 0 : 2;
+#pragma unroll
+            for (int kq = 0; kq < 2; ++kq) {
+                const int kc = kc0 + kq;
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int k = 32 * kc + 2 * e;
+                    w[e] = uint32_t(a1_value<N2>(P2, l, k)) | (uint32_t(a1_value<N2>(P2, l, k + 1)) << 16);
+                }
+                tmem_st_32x32b_x16(taddr + 16 * kc, w);
+            }
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        named_barrier_sync(3, kSetupThreads);
+        tc_fence_after();
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
     // Buffer hand-offs from the tensor pipe are commits by the MMA warp: stage 1
     // of a batch completing frees its x (and lo) tile and fills its D1 region;
     // stage 2 of a group completing fills a D2 region; stage 2 of a whole batch
@@ -491,9 +592,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int e = t + kXThreads * u;
                 const int c = e / (8 * N1), rem = e % (8 * N1), r = rem >> 3, up = rem & 7;
                 const int b0 = (N2 == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
+                const float4 ca = *reinterpret_cast<const float4 *>(cinv + r * N2 + b0);
+                const float4 cb = *reinterpret_cast<const float4 *>(cinv + r * N2 + b0 + 4);
+                const float cv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    const float c0 = cinv[r * N2 + b0 + 2 * p], c1 = cinv[r * N2 + b0 + 2 * p + 1];
+                    const float c0 = cv[2 * p], c1 = cv[2 * p + 1];
                     ch[u][p] = pack_bf16x2(c0, c1);
                     cl[u][p] = pack_bf16x2(c0 - __uint_as_float(ch[u][p] << 16),
                                            c1 - __uint_as_float(ch[u][p] & 0xFFFF0000u));
@@ -657,9 +761,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // exact quotients by a few ulps, far inside the rounding-boundary window
             const float s = alpha * m * (1.0f / 7.0f);
             const float inv = s > 0.0f ? fminf(__fdividef(1.0f, s), 3.0e38f) : 0.0f;
+            const uint64_t inv2 = uint64_t(__float_as_uint(inv)) | (uint64_t(__float_as_uint(inv)) << 32);
             unsigned char *stg = smem + C::OFF_STG + (2 * ew + buf) * C::STG;
-            // this thread's two bytes of every row: columns 4 g8 .. 4 g8 + 3 of the warp's 32
+            // this thread's two bytes of every row: columns 4 g8 .. 4 g8 + 3 of the warp's 32.
+            // It writes rows row0 + 16 c + 8 rep + 2 qq + d, whose swizzle term of
+            // stg_offset is the same for all of them: qq (64-byte rows; row0 is a
+            // multiple of 16) or qq >> 1 (32-byte rows).  So every store is one base
+            // address plus a constant.
             const int row0 = tok_h * N1, bcol = ((32 * q) % N2) / 2 + 2 * g8;
+            const int swz_t = N2 == 128 ? qq : (qq >> 1);
+            unsigned char *tbase = stg + (row0 + 2 * qq) * C::RB + ((((bcol >> 4) ^ swz_t) << 4) | (bcol & 15));
             const uint32_t t0 = tmem + (uint32_t(32 * q) << 16) + C::R2(int(b));
             constexpr int CB = N1 % 32 == 0 ? 2 : 1;  // 16-column chunks per load
 #pragma unroll
@@ -680,16 +791,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
 #pragma unroll
                 for (int rep = 0; rep < 2 * CB; ++rep) {
-                    const int i0 = 16 * c0 + 8 * rep + 2 * qq;
+                    // rows (i0, i0 + 1), i0 = 16 c0 + 8 rep + 2 qq, of: the even and odd
+                    // column of half 0, likewise half 1
+                    const uint64_t ea = round_codes2(ra[4 * rep], ra[4 * rep + 1], inv2);
+                    const uint64_t oa = round_codes2(ra[4 * rep + 2], ra[4 * rep + 3], inv2);
+                    const uint64_t eb = round_codes2(rb[4 * rep], rb[4 * rep + 1], inv2);
+                    const uint64_t ob = round_codes2(rb[4 * rep + 2], rb[4 * rep + 3], inv2);
 #pragma unroll
                     for (int d = 0; d < 2; ++d) {
                         // row i0 + d: columns 4 g8 + (0, 1) from half 0, + (2, 3) from half 1;
                         // byte = even column in the low nibble, odd in the high one
-                        const uint32_t wb = pack_s4x2(round_code(rb[4 * rep + 2 + d], inv, one),
-                                                      round_code(rb[4 * rep + d], inv, one), 0u);
-                        const uint32_t w = pack_s4x2(round_code(ra[4 * rep + 2 + d], inv, one),
-                                                     round_code(ra[4 * rep + d], inv, one), wb);
-                        *reinterpret_cast<uint16_t *>(stg + stg_offset<N2>(row0 + i0 + d, bcol)) = uint16_t(w);
+                        const int sh = 32 * d;
+                        const uint32_t wb = pack_s4x2(code_of(uint32_t(ob >> sh), one), code_of(uint32_t(eb >> sh), one), 0u);
+                        const uint32_t w = pack_s4x2(code_of(uint32_t(oa >> sh), one), code_of(uint32_t(ea >> sh), one), wb);
+                        *reinterpret_cast<uint16_t *>(tbase + (16 * c0 + 8 * rep + d) * C::RB) = uint16_t(w);
                     }
                 }
             }
