@@ -254,20 +254,17 @@ __device__ __forceinline__ void split2(uint64_t v, uint32_t &hi, uint32_t &lo) {
     lo = pack_bf16x2(__uint_as_float(uint32_t(l)), __uint_as_float(uint32_t(l >> 32)));
 }
 
-// round_half_even(y * inv) for two values at once, valid for |y * inv| < 2^22
-// (alpha >= 2^-19): adding 1.5 * 2^23 leaves the rounded integer in the low
-// mantissa bits of each fp32 result (bit patterns 0x4B400000 + k).
+// round_half_even(y * inv) as an int, valid for |y * inv| < 2^22 (alpha >= 2^-19):
+// adding 1.5 * 2^23 leaves the rounded integer in the low mantissa bits (bit
+// pattern 0x4B400000 + k).  The offset is removed by an integer multiply-add
+// with `one` (== 1, loaded at run time), which runs beside the floating-point
+// work instead of on the logic pipe.  (A packed fp32x2 form needs register
+// pairs the TMEM loads do not provide, and costs more instructions.)
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;  // 1.5 * 2^23
-__device__ __forceinline__ uint64_t round_codes2(uint32_t y0, uint32_t y1, uint64_t inv2) {
-    constexpr uint64_t magic2 = uint64_t(kRoundMagicBits) | (uint64_t(kRoundMagicBits) << 32);
-    return f32x2_fma(uint64_t(y0) | (uint64_t(y1) << 32), inv2, magic2);
-}
-// The integer k of one such result.  The offset is removed by an integer
-// multiply-add with `one` (== 1, loaded at run time), which runs beside the
-// floating-point work instead of on the logic pipe.
-__device__ __forceinline__ int code_of(uint32_t bits, int one) {
+__device__ __forceinline__ int round_code(uint32_t ybits, float inv, int one) {
+    const uint32_t b = __float_as_uint(fmaf(__uint_as_float(ybits), inv, 12582912.0f));
     int k;
-    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k) : "r"(bits), "r"(one), "r"(-int(kRoundMagicBits)));
+    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k) : "r"(b), "r"(one), "r"(-int(kRoundMagicBits)));
     return k;
 }
 
@@ -761,7 +758,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // exact quotients by a few ulps, far inside the rounding-boundary window
             const float s = alpha * m * (1.0f / 7.0f);
             const float inv = s > 0.0f ? fminf(__fdividef(1.0f, s), 3.0e38f) : 0.0f;
-            const uint64_t inv2 = uint64_t(__float_as_uint(inv)) | (uint64_t(__float_as_uint(inv)) << 32);
             unsigned char *stg = smem + C::OFF_STG + (2 * ew + buf) * C::STG;
             // this thread's two bytes of every row: columns 4 g8 .. 4 g8 + 3 of the warp's 32.
             // It writes rows row0 + 16 c + 8 rep + 2 qq + d, whose swizzle term of
@@ -791,19 +787,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
 #pragma unroll
                 for (int rep = 0; rep < 2 * CB; ++rep) {
-                    // rows (i0, i0 + 1), i0 = 16 c0 + 8 rep + 2 qq, of: the even and odd
-                    // column of half 0, likewise half 1
-                    const uint64_t ea = round_codes2(ra[4 * rep], ra[4 * rep + 1], inv2);
-                    const uint64_t oa = round_codes2(ra[4 * rep + 2], ra[4 * rep + 3], inv2);
-                    const uint64_t eb = round_codes2(rb[4 * rep], rb[4 * rep + 1], inv2);
-                    const uint64_t ob = round_codes2(rb[4 * rep + 2], rb[4 * rep + 3], inv2);
+                    // rows i0 + d, i0 = 16 c0 + 8 rep + 2 qq: registers 4 rep + d hold the even
+                    // column, 4 rep + 2 + d the odd one, of half 0 (ra) and half 1 (rb)
 #pragma unroll
                     for (int d = 0; d < 2; ++d) {
                         // row i0 + d: columns 4 g8 + (0, 1) from half 0, + (2, 3) from half 1;
                         // byte = even column in the low nibble, odd in the high one
-                        const int sh = 32 * d;
-                        const uint32_t wb = pack_s4x2(code_of(uint32_t(ob >> sh), one), code_of(uint32_t(eb >> sh), one), 0u);
-                        const uint32_t w = pack_s4x2(code_of(uint32_t(oa >> sh), one), code_of(uint32_t(ea >> sh), one), wb);
+                        const uint32_t wb = pack_s4x2(round_code(rb[4 * rep + 2 + d], inv, one),
+                                                      round_code(rb[4 * rep + d], inv, one), 0u);
+                        const uint32_t w = pack_s4x2(round_code(ra[4 * rep + 2 + d], inv, one),
+                                                     round_code(ra[4 * rep + d], inv, one), wb);
                         *reinterpret_cast<uint16_t *>(tbase + (16 * c0 + 8 * rep + d) * C::RB) = uint16_t(w);
                     }
                 }
