@@ -102,6 +102,34 @@ kq_status kq_dequant_inverse(const uint8_t *q, const float *scale, const float *
                              int n1, int n2, kq_stream_t stream);
 
 /*
+ * kq_w4a4_gemm -- the product that consumes the codes (FlatQuant page,
+ * "Kronecker factorization": Q(X P) Q(P^-1 W^T), the W4A4 linear layer):
+ *
+ *     y[m][o] = sx[m] * sw[o] * sum_k qx[m][k] * qw[o][k]
+ *
+ * qx      [M, K/2] device, packed INT4 activation codes, row-major, as written
+ *         by kq_transform_quant (element 2k in the low nibble of byte k,
+ *         two's complement); 16-byte aligned.
+ * sx      [M] device fp32, one scale per row of qx (kq_transform_quant's
+ *         scale_out).
+ * qw      [N, K/2] device, packed INT4 weight codes in the same layout: one
+ *         row per output channel, e.g. the weight rows transformed with
+ *         factors P1^-T, P2^-T and the channel vector c and quantised by
+ *         kq_transform_quant; 16-byte aligned.
+ * sw      [N] device fp32, one scale per output channel.
+ * y       [M, N] device fp32, row-major, written; must not overlap the inputs.
+ * K       multiple of 128 in [128, 262144] (every n = n1 n2 of kq_transform_quant);
+ *         M, N >= 0 (0 is a no-op).
+ * The integer sums are exact (|sum| <= 64 K < 2^24); y is (float(sum) * sx[m])
+ * * sw[o] in fp32.  The library allocates nothing; asynchronous on `stream`.
+ * Returns KQ_ERR_SHAPE for negative M/N or a K out of range, KQ_ERR_NULL,
+ * KQ_ERR_ALIGN, KQ_ERR_ARG for overlapping output, KQ_ERR_CUDA if the launch
+ * fails.
+ */
+kq_status kq_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw, float *y,
+                       int64_t M, int64_t N, int64_t K, kq_stream_t stream);
+
+/*
  * kq_device_error -- read and clear the device-side status word that the
  * kernels set when a bounded wait gives up (they then skip their remaining
  * work instead of hanging).  Synchronises `stream`.  *code receives 0 when

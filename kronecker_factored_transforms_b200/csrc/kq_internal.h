@@ -40,4 +40,8 @@ cudaError_t launch_dequant_inverse(const uint8_t *q, const float *scale, const f
                                    const float *P2inv, const float *c, float *x_hat, int64_t T,
                                    int n1, int n2, cudaStream_t stream);
 
+// W4A4 product of packed INT4 codes: y = sx[m] sw[o] sum_k qx[m][k] qw[o][k].
+cudaError_t launch_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw, float *y,
+                             int64_t M, int64_t N, int64_t K, int device, cudaStream_t stream);
+
 }  // namespace kq

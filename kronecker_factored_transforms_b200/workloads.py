@@ -201,3 +201,14 @@ def workload_bytes(T: int, n: int) -> int:
 def workload_flops(T: int, n1: int, n2: int) -> int:
     """Algorithmic flops of the factored contraction: 2 n (n1 + n2) per token."""
     return T * 2 * n1 * n2 * (n1 + n2)
+
+
+def make_weights(n: int, n_out: int, seed: int) -> np.ndarray:
+    """Synthetic linear-layer weight W [n_out, n] as bf16 bits: N(0, 1/n) entries
+    with 1% of the input channels (columns) scaled by 8, the way trained
+    weights carry a few large input channels.  Seeded; no method arithmetic."""
+    rng = np.random.default_rng([seed, 7919])
+    W = rng.standard_normal((n_out, n)) / np.sqrt(n)
+    cols = rng.choice(n, size=max(1, round(0.01 * n)), replace=False)
+    W[:, cols] *= 8.0
+    return f32_to_bf16_bits(W.astype(np.float32))

@@ -14,6 +14,8 @@ Parity status of each function (pins live in ``tests/test_oracle_pins.py``):
   transform_quant   pinned: equals quantize(transform(.)) exactly.
   dequant_inverse   pinned: round trip against numpy fp64 inverse of the
                     explicit Kronecker matrix.
+  w4a4_gemm         pinned: brute-force integer loops on small inputs,
+                    hand-derived extreme-code products, scale placement.
 """
 from __future__ import annotations
 
@@ -144,3 +146,18 @@ def unpack_codes(packed) -> np.ndarray:
     out[..., 0::2] = lo
     out[..., 1::2] = hi
     return out
+
+
+def w4a4_gemm(qx_packed, sx, qw_packed, sw) -> np.ndarray:
+    """The W4A4 product that consumes the codes (FlatQuant, "Kronecker
+    factorization": Q(X P) Q(P^-1 W^T)), in fp64:
+
+        y[m][o] = sx[m] * sw[o] * sum_k qx[m][k] * qw[o][k]
+
+    qx [M, K/2] and qw [N, K/2] packed INT4 (as unpack_codes), sx [M], sw [N]
+    fp32.  The integer sum is formed exactly (a float64 matrix product of small
+    integers: every partial sum is an integer far below 2^53)."""
+    qx = unpack_codes(qx_packed).astype(np.float64)
+    qw = unpack_codes(qw_packed).astype(np.float64)
+    acc = qx @ qw.T
+    return acc * np.asarray(sx, dtype=np.float64)[:, None] * np.asarray(sw, dtype=np.float64)[None, :]

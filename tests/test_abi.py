@@ -29,7 +29,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for must in ("kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_status_string",
-                 "kq_kernel_name", "kq_device_error", "kq_version"):
+                 "kq_kernel_name", "kq_device_error", "kq_version", "kq_w4a4_gemm"):
         assert must in names
 
 
@@ -110,6 +110,24 @@ def test_dequant_inverse_validation(kq):
     assert f(Q + 1, S, P1, P2, None, Y, 4, 16, 16, None) == kq.KQ_ERR_ALIGN
     assert f(Q, S, P1, P2, None, Q + 32, 4, 16, 16, None) == kq.KQ_ERR_ARG
     assert f(None, None, None, None, None, None, 0, 16, 16, None) == kq.KQ_OK
+
+
+def test_w4a4_gemm_validation(kq):
+    f = kq.lib.kq_w4a4_gemm
+    # qx [4, 64], sx [4], qw [8, 64], sw [8], y [4, 8]: fake, well separated, aligned addresses
+    qx, sx, qw, sw, y = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+    assert f(qx, sx, qw, sw, y, -1, 8, 128, None) == kq.KQ_ERR_SHAPE
+    assert f(qx, sx, qw, sw, y, 4, -1, 128, None) == kq.KQ_ERR_SHAPE
+    for bad_k in (0, 64, 100, 192, 262144 + 128):
+        assert f(qx, sx, qw, sw, y, 4, 8, bad_k, None) == kq.KQ_ERR_SHAPE, bad_k
+    assert f(qx, None, qw, sw, y, 4, 8, 128, None) == kq.KQ_ERR_NULL
+    assert f(qx + 8, sx, qw, sw, y, 4, 8, 128, None) == kq.KQ_ERR_ALIGN
+    assert f(qx, sx, qw + 4, sw, y, 4, 8, 128, None) == kq.KQ_ERR_ALIGN
+    assert f(qx, sx + 2, qw, sw, y, 4, 8, 128, None) == kq.KQ_ERR_ALIGN
+    assert f(qx, sx, qw, sw, qx + 64, 4, 8, 128, None) == kq.KQ_ERR_ARG   # y overlaps qx
+    assert f(qx, sx, qw, sw, sw, 4, 8, 128, None) == kq.KQ_ERR_ARG        # y overlaps sw
+    assert f(None, None, None, None, None, 0, 8, 128, None) == kq.KQ_OK   # empty: no-op
+    assert f(None, None, None, None, None, 4, 0, 128, None) == kq.KQ_OK
 
 
 def test_device_error_rejects_null(kq):
