@@ -7,147 +7,251 @@
 // the low nibble of byte k (the layout kq_transform_quant writes), sx [M] and
 // sw [N] the per-token and per-output-channel fp32 scales, y [M, N] fp32.
 //
-// Tensor cores read the nibbles as they are: mma.sync m16n8k64 with s4
-// operands and s32 accumulators (the sum is exact), fed by ldmatrix from a
-// 4-stage cp.async ring.  Tile 128 x 128 x 128 per CTA, 8 warps of 64 x 32.
-// The integer sum is converted to fp32 (exact: |sum| <= 64 K < 2^24) and
-// multiplied by sx[m], then by sw[o].
+// The 5th-generation tensor cores have no 4-bit integer kind, so each 128-code
+// K chunk goes: packed tiles by TMA -> eight expander warps widen every code q
+// to the int8 16 q (a mask keeps the high nibble where it is, a shift moves the
+// low one up) -> tcgen05.mma kind::i8 (s8 x s8 -> s32 in TMEM).  Within every
+// 8-code group the expanders write the even codes before the odd ones, the
+// same way for both operands, which leaves every dot product unchanged.  The
+// s32 sums are 256 times the code sums and exact (|sum| <= 16384 K < 2^31); the
+// epilogue shifts the factor out and applies (float(sum) * sx[m]) * sw[o].
+//
+// One CTA per 128 x 256 output tile.  Warps: 0 TMA producer | 1 TMEM
+// allocator + MMA issuer | 4-11 expanders, then the epilogue | 2-3 idle.
+// Every mbarrier wait is bounded (kq_wait.cuh).
 #include <mutex>
 
 #include "kq_common.cuh"
 #include "kq_internal.h"
+#include "kq_tc05_ptx.cuh"
+#include "kq_wait.cuh"
 
 namespace kq {
 namespace {
 
-constexpr int BM = 128, BN = 128;      // tile rows (tokens) and columns (output channels)
-constexpr int BKB = 64;                // K bytes per stage (128 codes)
-constexpr int STAGES = 4;
-constexpr int GEMM_THREADS = 256;      // 8 warps: 2 along M x 4 along N, 64 x 32 each
-constexpr int STAGE_BYTES = (BM + BN) * BKB;
-constexpr int GEMM_SMEM = STAGES * STAGE_BYTES;
+using namespace tc;
 
-// Rows of 64 bytes (four 16-byte chunks); chunk c of row r is stored at chunk
-// c ^ ((r >> 1) & 3), so the eight rows an ldmatrix reads hit 32 distinct banks.
-__device__ __forceinline__ uint32_t tile_off(int r, int chunk) {
-    return uint32_t(r * BKB + ((chunk ^ ((r >> 1) & 3)) << 4));
+constexpr int TM = 128, TN = 256, KC = 128;            // tile rows, columns, codes per K chunk
+constexpr int PA = TM * KC / 2, PB = TN * KC / 2;       // packed bytes per chunk: 8 KB, 16 KB
+constexpr int EA = TM * KC, EB = TN * KC;               // widened int8 bytes per chunk: 16 KB, 32 KB
+constexpr int NS = 4, NE = 2;                           // packed stages, widened stages
+constexpr int G_THREADS = 384;                          // 12 warps
+constexpr int XW0 = 4, NXW = 8;                         // expander / epilogue warps 4-11
+constexpr int OFF_E = NS * (PA + PB);                   // 96 KB: widened stages (1024-aligned)
+constexpr int OFF_BAR = OFF_E + NE * (EA + EB);
+constexpr int FULL = 0, EMPTY = NS, XFULL = 2 * NS, XEMPTY = 2 * NS + NE, DONE = 2 * NS + 2 * NE;
+constexpr int NBAR = DONE + 1;
+constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;            // TMEM base, abort flag
+constexpr int G_SMEM = OFF_MISC + 16 + 1024;            // + slack for 1024-byte alignment
+constexpr uint32_t TMEM_COLS = TN;                      // s32 accumulator: 256 columns
+static_assert(OFF_E % 1024 == 0 && (EA + EB) % 1024 == 0 && EA % 1024 == 0, "swizzle atoms");
+static_assert(G_SMEM <= 227 * 1024, "shared memory budget");
+
+enum : unsigned { kSiteGemm = 64u };
+
+// Instruction descriptor: signed int8 A and B (K-major), s32 accumulator, M x N.
+__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
+    return (2u << 4)                      // accumulator format: s32
+           | (1u << 7)                    // A format: signed 8-bit
+           | (1u << 10)                   // B format: signed 8-bit
+           | (uint32_t(N >> 3) << 17)     // N / 8
+           | (uint32_t(M >> 4) << 24);    // M / 16
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
+// D (+)= A B^T with both operands in shared memory, described by the low
+// halves of their 128B-swizzle descriptors.
+template <int ACC>
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\tmov.b64 ad, {%1, %3};\n\tmov.b64 bd, {%2, %3};\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], ad, bd, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(kSdescSw128Hi), "r"(idesc), "n"(ACC)
+        : "memory");
 }
 
-__device__ __forceinline__ void mma_s4(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile("mma.sync.aligned.m16n8k64.row.col.s32.s4.s4.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-                 "{%0,%1,%2,%3};"
-                 : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
+// Byte offset of the 16-byte chunk `c` of row `r` in a 128B-swizzled K-major tile.
+__device__ __forceinline__ uint32_t sw128_chunk(int r, int c) { return uint32_t(r * 128 + ((c ^ (r & 7)) << 4)); }
 
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-    kq_w4a4_gemm_kernel(const uint8_t *__restrict__ qx, const float *__restrict__ sx,
-                        const uint8_t *__restrict__ qw, const float *__restrict__ sw, float *__restrict__ y,
-                        int64_t M, int64_t N, int64_t K) {
-    extern __shared__ __align__(128) unsigned char gsm[];
-    const uint32_t sbase = smem_u32(gsm);
+__global__ void __launch_bounds__(G_THREADS, 1)
+    kq_w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                      const float *__restrict__ sx, const float *__restrict__ sw, float *__restrict__ y,
+                      int64_t M, int64_t N, int64_t K, unsigned int *err) {
+    extern __shared__ __align__(1024) unsigned char gsm_raw[];
+    const uint32_t raw_addr = smem_u32(gsm_raw);
+    const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+    unsigned char *smem = gsm_raw + (sbase - raw_addr);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wm = warp >> 2, wn = warp & 3;
-    const int64_t m0 = int64_t(blockIdx.y) * BM, n0 = int64_t(blockIdx.x) * BN;
-    const int64_t kbytes = K / 2;
-    const int KT = int(K / (2 * BKB));
+    const int64_t m0 = int64_t(blockIdx.y) * TM, n0 = int64_t(blockIdx.x) * TN;
+    const int KT = int(K / KC);
+    auto bar = [&](int i) -> uint32_t { return sbase + uint32_t(OFF_BAR + 8 * i); };
+    volatile int *s_abort = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
 
-    // Each thread copies two 16-byte chunks of A and two of B per stage.
-    auto load_stage = [&](int kt, int slot) {
-        const uint32_t sa = sbase + uint32_t(slot * STAGE_BYTES), sb = sa + BM * BKB;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int c = tid + h * GEMM_THREADS, r = c >> 2, ch = c & 3;
-            const int64_t ga = m0 + r, gb = n0 + r;
-            const bool va = ga < M, vb = gb < N;
-            // rows past the end read nothing (size 0) and the chunk is zero-filled
-            const uint8_t *pa = qx + (va ? ga : 0) * kbytes + int64_t(kt) * BKB + ch * 16;
-            const uint8_t *pb = qw + (vb ? gb : 0) * kbytes + int64_t(kt) * BKB + ch * 16;
-            cp_async16(sa + tile_off(r, ch), pa, va);
-            cp_async16(sb + tile_off(r, ch), pb, vb);
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bar(FULL + s), 1);
+            mbar_init(bar(EMPTY + s), NXW);  // one arrive per expander warp
         }
-    };
+        for (int e = 0; e < NE; ++e) {
+            mbar_init(bar(XFULL + e), NXW);
+            mbar_init(bar(XEMPTY + e), 1);
+        }
+        mbar_init(bar(DONE), 1);
+        *s_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmap_a);
+        prefetch_tensormap(&tmap_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(sbase + OFF_MISC, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + OFF_MISC);
 
-    int acc[4][4][4];
+    if (warp == 0) {
+        // ---------------- TMA producer: packed A and B tiles of each K chunk ----------------
+        Ring r;
+        int issued = 0;
+        for (int kt = 0; kt < KT; ++kt, r.next(NS)) {
+            const bool ok = wait_bounded_err(bar(EMPTY + r.idx), r.phase ^ 1u, s_abort, kSiteGemm, kWaitLimitNs,
+                                             false, err);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            if (elect_one()) {
+                const uint32_t dst = sbase + uint32_t(r.idx * (PA + PB));
+                mbar_arrive_expect_tx(bar(FULL + r.idx), PA + PB);
+                tma_load_2d(dst, &tmap_a, kt * (KC / 2), int(m0), bar(FULL + r.idx));
+                tma_load_2d(dst + PA, &tmap_b, kt * (KC / 2), int(n0), bar(FULL + r.idx));
+            }
+            __syncwarp();
+            ++issued;
+        }
+        // every load issued has landed before the CTA can exit
+        Ring rd;
+        for (int i = 0; i < issued; ++i, rd.next(NS))
+            if (i + NS >= issued)
+                wait_bounded_err(bar(FULL + rd.idx), rd.phase, s_abort, kSiteGemm, kWaitLimitNs, true, err);
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        constexpr uint32_t idesc = idesc_s8_s32(TM, TN);
+        Ring r;
+        for (int kt = 0; kt < KT; ++kt, r.next(NE)) {
+            const bool ok = wait_bounded_err(bar(XFULL + r.idx), r.phase, s_abort, kSiteGemm, kWaitLimitNs, false,
+                                             err);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const uint32_t ea = sbase + uint32_t(OFF_E + r.idx * (EA + EB));
+            const uint32_t al = sdesc_sw128_lo(ea), bl = sdesc_sw128_lo(ea + EA);
+            if (elect_one()) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+                for (int kk = 0; kk < KC / 32; ++kk) {  // K = 32 int8 per MMA: +32 bytes
+                    if ((kt | kk) != 0)
+                        mma_i8<1>(tmem, al + 2 * kk, bl + 2 * kk, idesc);
+                    else
+                        mma_i8<0>(tmem, al + 2 * kk, bl + 2 * kk, idesc);
+                }
+                tc_commit(bar(XEMPTY + r.idx));  // widened stage free once these MMAs complete
+            }
+            __syncwarp();
+        }
+        // DONE completes once every MMA this thread issued has completed
+        if (elect_one()) tc_commit(bar(DONE));
+        __syncwarp();
+        wait_bounded_err(bar(DONE), 0u, s_abort, kSiteGemm, kWaitLimitNs, true, err);
+        __syncwarp();
+    } else if (warp >= XW0 && warp < XW0 + NXW) {
+        // ---------------- expanders: packed INT4 -> int8 (x16), swizzled K-major ----------------
+        const int xt = tid - XW0 * 32;                // 0 .. 255
+        constexpr int UNITS = (TM + TN) * (KC / 32);  // 16-byte packed units per chunk: 1536
+        constexpr int UPT = UNITS / (NXW * 32);       // 6 per thread
+        static_assert(UNITS % (NXW * 32) == 0, "unit split");
+        Ring rs, re;
+        bool ok = true;
+        for (int kt = 0; kt < KT; ++kt, rs.next(NS), re.next(NE)) {
+            ok = wait_bounded_err(bar(FULL + rs.idx), rs.phase, s_abort, kSiteGemm, kWaitLimitNs, false, err);
+            ok = ok && wait_bounded_err(bar(XEMPTY + re.idx), re.phase ^ 1u, s_abort, kSiteGemm, kWaitLimitNs,
+                                        false, err);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const unsigned char *pk = smem + rs.idx * (PA + PB);
+            unsigned char *ex = smem + OFF_E + re.idx * (EA + EB);
+            uint4 v[UPT];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+            for (int i = 0; i < UPT; ++i) {
+                const int u = xt + i * NXW * 32;  // A units first (row u / 4), then B
+                v[i] = *reinterpret_cast<const uint4 *>(pk + u * 16);
+            }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[i][j][e] = 0;
-
+            for (int i = 0; i < UPT; ++i) {
+                const int u = xt + i * NXW * 32;
+                const bool isb = u >= TM * (KC / 32);
+                const int ub = isb ? u - TM * (KC / 32) : u;
+                const int r = ub >> 2, q = ub & 3;  // row, 16-byte unit within the row's 64 packed bytes
+                unsigned char *dst = ex + (isb ? EA : 0);
+                const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+                uint32_t o[8];
 #pragma unroll
-    for (int s = 0; s < STAGES - 1; ++s) {
-        if (s < KT) load_stage(s, s);
-        cp_async_commit();
+                for (int j = 0; j < 4; ++j) {
+                    o[2 * j] = (w[j] << 4) & 0xF0F0F0F0u;  // even codes of the 8-code group, x16
+                    o[2 * j + 1] = w[j] & 0xF0F0F0F0u;     // odd codes, x16
+                }
+                *reinterpret_cast<uint4 *>(dst + sw128_chunk(r, 2 * q)) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4 *>(dst + sw128_chunk(r, 2 * q + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+            fence_proxy_async_smem();  // widened tile visible to the tensor cores
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(EMPTY + rs.idx));  // packed stage read
+                mbar_arrive(bar(XFULL + re.idx));  // widened stage written
+            }
+        }
+        // ---------------- epilogue: TMEM -> scales -> y ----------------
+        const bool done = wait_bounded_err(bar(DONE), 0u, s_abort, kSiteGemm, kWaitLimitNs, false, err);
+        if (__all_sync(0xffffffffu, done && ok)) {
+            tc_fence_after();
+            const int q = warp & 3, h = (warp - XW0) >> 2;  // lane quarter, column half
+            const int64_t m = m0 + 32 * q + lane;
+            const float fx = m < M ? sx[m] : 0.0f;
+            float *yrow = y + (m < M ? m : 0) * N;
+            // 16-byte stores only where every row start is 16-byte aligned
+            const bool vec = (N % 4) == 0 && (reinterpret_cast<uintptr_t>(y) & 15) == 0;
+#pragma unroll 1
+            for (int c = 0; c < TN / 2 / 32; ++c) {
+                uint32_t a[32];
+                tmem_ld_32x32b_x32(tmem + (uint32_t(32 * q) << 16) + uint32_t(128 * h + 32 * c), a);
+                tmem_wait_ld();
+                const int64_t nb = n0 + 128 * h + 32 * c;
+                if (m < M) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        const int64_t n = nb + e;
+                        float r4[4];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            r4[t] = (float(int(a[e + t]) >> 8) * fx) * (n + t < N ? sw[n + t] : 0.0f);
+                        if (vec && n + 3 < N) {
+                            *reinterpret_cast<float4 *>(yrow + n) = make_float4(r4[0], r4[1], r4[2], r4[3]);
+                        } else {
+#pragma unroll
+                            for (int t = 0; t < 4; ++t)
+                                if (n + t < N) yrow[n + t] = r4[t];
+                        }
+                    }
+                }
+            }
+        }
     }
 
-    // ldmatrix row addresses: thread t serves matrix t / 8, row t % 8
-    const int mat = lane >> 3, mr = lane & 7;
-    for (int kt = 0; kt < KT; ++kt) {
-        cp_async_wait<STAGES - 2>();
-        __syncthreads();  // tile kt landed for everyone; slot (kt - 1) % STAGES is free
-        if (kt + STAGES - 1 < KT) load_stage(kt + STAGES - 1, (kt + STAGES - 1) % STAGES);
-        cp_async_commit();
-
-        const uint32_t sa = sbase + uint32_t((kt % STAGES) * STAGE_BYTES), sb = sa + BM * BKB;
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {  // two k64 steps per stage
-            uint32_t a[4][4], b[4][2];
-#pragma unroll
-            for (int mt = 0; mt < 4; ++mt) {
-                // matrices: rows +0 / +8 of the m16 tile, bytes [0,16) / [16,32) of the k64 step
-                const int r = wm * 64 + mt * 16 + (mat & 1) * 8 + mr;
-                ldmatrix_x4(sa + tile_off(r, 2 * kk + (mat >> 1)), a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
-            }
-#pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                // matrices: n8 tile 2 np (k halves 0, 1), then n8 tile 2 np + 1
-                const int r = wn * 32 + (2 * np + (mat >> 1)) * 8 + mr;
-                ldmatrix_x4(sb + tile_off(r, 2 * kk + (mat & 1)), b[2 * np][0], b[2 * np][1], b[2 * np + 1][0],
-                            b[2 * np + 1][1]);
-            }
-#pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) mma_s4(acc[mt][nt], a[mt], b[nt][0], b[nt][1]);
-        }
-    }
-    cp_async_wait<0>();
-
-    // epilogue: accumulator (row g (+8), columns 2 tig, 2 tig + 1) of each m16n8 tile
-    const int g = lane >> 2, tig = lane & 3;
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt) {
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const int64_t m = m0 + wm * 64 + mt * 16 + g + 8 * hr;
-            if (m >= M) continue;
-            const float fx = sx[m];
-            float *yrow = y + m * N;
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const int64_t n = n0 + wn * 32 + nt * 8 + 2 * tig;
-                if (n < N) yrow[n] = (float(acc[mt][nt][2 * hr]) * fx) * sw[n];
-                if (n + 1 < N) yrow[n + 1] = (float(acc[mt][nt][2 * hr + 1]) * fx) * sw[n + 1];
-            }
-        }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
@@ -159,12 +263,31 @@ cudaError_t launch_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *
     static cudaError_t attr_err[64];
     if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[device], [&] {
-        attr_err[device] = cudaFuncSetAttribute(kq_w4a4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                GEMM_SMEM);
+        attr_err[device] = cudaFuncSetAttribute(kq_w4a4_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                G_SMEM);
     });
     if (attr_err[device] != cudaSuccess) return attr_err[device];
-    const dim3 grid(unsigned((N + BN - 1) / BN), unsigned((M + BM - 1) / BM));
-    kq_w4a4_gemm_kernel<<<grid, GEMM_THREADS, GEMM_SMEM, stream>>>(qx, sx, qw, sw, y, M, N, K);
+    unsigned int *err = nullptr;
+    cudaError_t e = device_error_word(device, &err);
+    if (e != cudaSuccess) return e;
+    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (!encode) return cudaErrorNotSupported;
+    // packed codes: rows of K/2 bytes; one box = one K chunk (64 bytes) of TM or TN rows
+    CUtensorMap ta, tb;
+    const cuuint64_t da[2] = {cuuint64_t(K / 2), cuuint64_t(M)}, db[2] = {cuuint64_t(K / 2), cuuint64_t(N)};
+    const cuuint64_t stride[1] = {cuuint64_t(K / 2)};
+    const cuuint32_t boxa[2] = {cuuint32_t(KC / 2), cuuint32_t(TM)}, boxb[2] = {cuuint32_t(KC / 2), cuuint32_t(TN)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = encode(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(qx), da, stride, boxa, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    r = encode(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(qw), db, stride, boxb, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    const dim3 grid(unsigned((N + TN - 1) / TN), unsigned((M + TM - 1) / TM));
+    kq_w4a4_tc_kernel<<<grid, G_THREADS, G_SMEM, stream>>>(ta, tb, sx, sw, y, M, N, K, err);
     return cudaGetLastError();
 }
 

@@ -1,6 +1,8 @@
 // kq_internal.h -- launch plumbing shared between the C ABI and the kernels.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -31,6 +33,12 @@ cudaError_t launch_tc05(const LaunchArgs &a);
 
 // Diagnostic: a kernel whose bounded wait on a never-signalled barrier gives up.
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
+
+// cuTensorMapEncodeTiled from the driver (null if unavailable).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// Device address of the status word (for kernels in other translation units).
+cudaError_t device_error_word(int device, unsigned int **word);
 
 // Read and clear the device status word set by bounded waits that gave up.
 cudaError_t read_and_clear_device_error(cudaStream_t stream, unsigned int *code);

@@ -42,11 +42,26 @@
 #include "kq_common.cuh"
 #include "kq_internal.h"
 #include "kq_tc05_ptx.cuh"
+#include "kq_wait.cuh"
 
 namespace kq {
 
 // Nonzero when a bounded wait gave up; each site ORs its own bit.
 __device__ unsigned int g_device_error = 0;
+
+cudaError_t device_error_word(int device, unsigned int **word) {
+    static std::once_flag once[64];
+    static unsigned int *addr[64];
+    static cudaError_t err[64];
+    if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+    std::call_once(once[device], [&] {
+        void *p = nullptr;
+        err[device] = cudaGetSymbolAddress(&p, g_device_error);
+        addr[device] = static_cast<unsigned int *>(p);
+    });
+    *word = addr[device];
+    return err[device];
+}
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, unsigned int *code) {
     static const unsigned int zero = 0;
@@ -83,8 +98,6 @@ __device__ __forceinline__ int xsplit_index(int warp) {
     default: return -1;
     }
 }
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // about one second
-
 enum : unsigned {
     kSiteProducer = 1u,
     kSiteXSplit = 2u,
@@ -95,29 +108,10 @@ enum : unsigned {
     kSiteSelfTest = 256u,
 };
 
-// Wait for the phase of parity `parity` of mbarrier `bar` to complete, for at
-// most `limit_ns`.  Returns false (after flagging `site`) on timeout, or when
-// another role already aborted (unless `ignore_abort`).  Out of line: only
-// reached when the phase is not complete at the first look.
-__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int *abort, unsigned site,
-                                       uint64_t limit_ns, bool ignore_abort) {
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 31u) == 0) {
-            if (!ignore_abort && *abort) return false;
-            if (globaltimer_ns() - t0 > limit_ns) {
-                atomicOr(&g_device_error, site);
-                *abort = 1;
-                return false;
-            }
-        }
-    }
-}
+// Bounded waits (kq_wait.cuh) reporting through g_device_error.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int *abort,
                                              unsigned site, uint64_t limit_ns, bool ignore_abort) {
-    if (mbar_try_wait(bar, parity)) return true;
-    return wait_slow(bar, parity, abort, site, limit_ns, ignore_abort);
+    return wait_bounded_err(bar, parity, abort, site, limit_ns, ignore_abort, &g_device_error);
 }
 
 __host__ __device__ constexpr int align_up(int v, int a) { return (v + a - 1) / a * a; }
@@ -268,17 +262,6 @@ __device__ __forceinline__ int round_code(uint32_t ybits, float inv, int one) {
     return k;
 }
 
-// Position in a ring of n barrier-guarded slots: slot index and the parity of
-// the slot's current phase; advancing past the last slot flips the parity.
-struct Ring {
-    uint32_t idx = 0, phase = 0;
-    __device__ __forceinline__ void next(uint32_t n) {
-        if (++idx == n) {
-            idx = 0;
-            phase ^= 1u;
-        }
-    }
-};
 
 template <int N1, int N2, bool SCALED>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -837,19 +820,6 @@ __global__ void kq_selftest_wait_kernel(uint64_t limit_ns) {
 // ---------------------------------------------------------------------------
 // Host side.
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
 template <int N1, int N2, bool SCALED>
 cudaError_t launch_inst(const LaunchArgs &a) {
     using C = Cfg<N1, N2, SCALED>;
@@ -862,7 +832,7 @@ cudaError_t launch_inst(const LaunchArgs &a) {
     });
     if (attr_err[a.device] != cudaSuccess) return attr_err[a.device];
 
-    PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
+    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
     if (!encode) return cudaErrorNotSupported;
     CUtensorMap tmap;
     const cuuint64_t dims[2] = {cuuint64_t(N2), cuuint64_t(a.T) * N1};
@@ -912,6 +882,19 @@ cudaError_t dispatch_n1(const LaunchArgs &a) {
 }
 
 }  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
 
 bool tc05_supports(int n1, int n2, bool scaled) {
     if (n2 != 64 && n2 != 128) return false;
