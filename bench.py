@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["transform", "gemm"], default="transform",
+                    help="transform: the fused transform + INT4 path (default); gemm: the W4A4 product "
+                         "of packed codes that consumes it (M = N = K = 8192)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0,
@@ -237,10 +240,55 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------
 
+def run_gemm(args):
+    """The W4A4 product y = sx sw (qx qw^T) of a hidden-8192 layer: M tokens x
+    N output channels x K = n, packed INT4 codes in, fp32 out.  One step is one
+    kq_w4a4_gemm call; ops = 2 M N K.  Single GPU only."""
+    import torch
+    from kronecker_factored_transforms_b200 import _lib
+    M = N = K = 8192
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(8192)
+    qx = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
+    qw = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
+    sx = torch.rand(M, device=dev, generator=g)
+    sw = torch.rand(N, device=dev, generator=g)
+    y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        _lib.kq_w4a4_gemm(qx, sx, qw, sw, y, M, N, K, stream=stream.cuda_stream)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(0)
+    with sampler:
+        e0.record(stream)
+        for _ in range(args.steps):
+            _lib.kq_w4a4_gemm(qx, sx, qw, sw, y, M, N, K, stream=stream.cuda_stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    tops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+    hbm_peak, tf_peak, kind = measured_peaks()
+    int8_peak = 2.0 * tf_peak  # dense int8 runs at twice the bf16 rate
+    line = {"metric": "TOPS of the W4A4 product of packed INT4 codes (M = N = K = 8192)", "value": tops,
+            "unit": "TOPS", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4 (int8 MMA)",
+            "data": "synthetic", "config": {"workload": "w4a4 gemm M=N=K=8192, random codes and scales",
+                                             "M": M, "N": N, "K": K},
+            "roofline": {"bound": "tensor", "achieved": tops, "peak": int8_peak, "unit": "TOP/s",
+                         "frac": tops / int8_peak, "traffic": None,
+                         "peak_source": "2 x %s bf16 TF/s (int8 dense rate)" % kind},
+            "gpu_launches": args.steps, "clocks": sampler.report()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "gemm":
+        return run_gemm(args)
 
     import torch
     import torch.distributed as dist
