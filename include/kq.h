@@ -130,6 +130,30 @@ kq_status kq_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, co
                        int64_t M, int64_t N, int64_t K, kq_stream_t stream);
 
 /*
+ * kq_headwise_transform_quant -- the per-head transform of the key / value
+ * cache (FlatQuant page: P_h and P_v keep their full per-head shape; keys and
+ * values are transformed per head and quantised before storage).  For every
+ * token t and head h, the row x[t, h, :] of head_dim values is multiplied by
+ * the full factor Ph and quantised on its own with the INT4 rule of
+ * kq_transform_quant (s = alpha * max|y| / 7, round half to even, clamp to
+ * [-8, 7], two codes per byte, element 2k in the low nibble).
+ *
+ * x         [T, heads * head_dim] device bf16, row-major (head-major within a
+ *           token), 16-byte aligned.
+ * Ph        [head_dim, head_dim] device bf16, row-major, 16-byte aligned.
+ * alpha     clip ratio in [2^-19, 1].
+ * q_out     [T, heads * head_dim / 2] device uint8, 16-byte aligned, written.
+ * scale_out [T, heads] device fp32, written (0 for an all-zero row).
+ * head_dim  64 or 128; heads >= 1 (any count, e.g. 8 grouped-query heads);
+ *           T * heads < 2^31.
+ * Returns KQ_ERR_SHAPE, KQ_ERR_UNSUPPORTED (head_dim, or alpha below 2^-19),
+ * KQ_ERR_ARG (alpha outside (0, 1], overlapping buffers), KQ_ERR_NULL,
+ * KQ_ERR_ALIGN, KQ_ERR_CUDA.  Asynchronous on `stream`; allocates nothing.
+ */
+kq_status kq_headwise_transform_quant(const uint16_t *x, const uint16_t *Ph, float alpha, uint8_t *q_out,
+                                      float *scale_out, int64_t T, int heads, int head_dim, kq_stream_t stream);
+
+/*
  * kq_device_error -- read and clear the device-side status word that the
  * kernels set when a bounded wait gives up (they then skip their remaining
  * work instead of hanging).  Synchronises `stream`.  *code receives 0 when

@@ -42,8 +42,9 @@ def _load() -> ctypes.CDLL:
     lib.kq_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
     lib.kq_selftest_bounded_wait.argtypes = [I64, P]
     lib.kq_w4a4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P]
+    lib.kq_headwise_transform_quant.argtypes = [P, P, F32, P, P, I64, I32, I32, P]
     for f in (lib.kq_transform_quant, lib.kq_transform, lib.kq_dequant_inverse, lib.kq_device_error,
-              lib.kq_selftest_bounded_wait, lib.kq_w4a4_gemm):
+              lib.kq_selftest_bounded_wait, lib.kq_w4a4_gemm, lib.kq_headwise_transform_quant):
         f.restype = ctypes.c_int
     lib.kq_status_string.argtypes = [I32]
     lib.kq_status_string.restype = ctypes.c_char_p
@@ -57,7 +58,8 @@ def _load() -> ctypes.CDLL:
 lib = _load()
 
 EXPORTED = ("kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_device_error",
-            "kq_selftest_bounded_wait", "kq_status_string", "kq_kernel_name", "kq_version", "kq_w4a4_gemm")
+            "kq_selftest_bounded_wait", "kq_status_string", "kq_kernel_name", "kq_version", "kq_w4a4_gemm",
+            "kq_headwise_transform_quant")
 
 
 def _ptr(t) -> Optional[int]:
@@ -88,6 +90,13 @@ def kq_transform_quant(x, P1, P2, cinv, alpha: float, q_out, scale_out, T: int, 
     _check("kq_transform_quant",
            lib.kq_transform_quant(_ptr(x), _ptr(P1), _ptr(P2), _ptr(cinv), float(alpha), _ptr(q_out),
                                   _ptr(scale_out), int(T), int(n1), int(n2), _stream(stream)))
+
+
+def kq_headwise_transform_quant(x, Ph, alpha: float, q_out, scale_out, T: int, heads: int, head_dim: int,
+                                stream=None) -> None:
+    _check("kq_headwise_transform_quant",
+           lib.kq_headwise_transform_quant(_ptr(x), _ptr(Ph), float(alpha), _ptr(q_out), _ptr(scale_out), int(T),
+                                           int(heads), int(head_dim), _stream(stream)))
 
 
 def kq_w4a4_gemm(qx, sx, qw, sw, y, M: int, N: int, K: int, stream=None) -> None:

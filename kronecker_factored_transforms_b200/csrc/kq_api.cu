@@ -181,6 +181,31 @@ kq_status kq_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, co
     return err == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;
 }
 
+kq_status kq_headwise_transform_quant(const uint16_t *x, const uint16_t *Ph, float alpha, uint8_t *q_out,
+                                      float *scale_out, int64_t T, int heads, int head_dim, kq_stream_t stream) {
+    if (T < 0 || heads <= 0 || head_dim <= 0) return KQ_ERR_SHAPE;
+    if (head_dim != 64 && head_dim != 128) return KQ_ERR_UNSUPPORTED;
+    if (T > (int64_t(1) << 31) / heads) return KQ_ERR_SHAPE;  // rows are TMA coordinates
+    kq_status st = check_alpha(alpha);
+    if (st != KQ_OK) return st;
+    if (!(alpha >= 0x1p-19f)) return KQ_ERR_UNSUPPORTED;  // the code rounding's range
+    if (T == 0) return KQ_OK;
+    if (!x || !Ph || !q_out || !scale_out) return KQ_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(Ph, 16) || !aligned(q_out, 16) || !aligned(scale_out, 4)) return KQ_ERR_ALIGN;
+    const int64_t R = T * heads;
+    const Range in[2] = {range_of(x, uint64_t(R) * head_dim * 2), range_of(Ph, uint64_t(head_dim) * head_dim * 2)};
+    const Range out[2] = {range_of(q_out, uint64_t(R) * head_dim / 2), range_of(scale_out, uint64_t(R) * 4)};
+    for (const Range &o : out)
+        for (const Range &i : in)
+            if (overlap(o, i)) return KQ_ERR_ARG;
+    if (overlap(out[0], out[1])) return KQ_ERR_ARG;
+    DeviceInfo info;
+    if ((st = device_info(info)) != KQ_OK) return st;
+    cudaError_t err = kq::launch_rowwise(x, Ph, alpha, q_out, scale_out, R, head_dim, info.num_sms, info.device,
+                                         reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;
+}
+
 kq_status kq_device_error(kq_stream_t stream, int *code) {
     if (!code) return KQ_ERR_NULL;
     unsigned int v = 0;

@@ -52,4 +52,8 @@ cudaError_t launch_dequant_inverse(const uint8_t *q, const float *scale, const f
 cudaError_t launch_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw, float *y,
                              int64_t M, int64_t N, int64_t K, int device, cudaStream_t stream);
 
+// Per-head transform + INT4 per row: rows of head_dim (64 or 128) values.
+cudaError_t launch_rowwise(const uint16_t *x, const uint16_t *Ph, float alpha, uint8_t *q_out, float *scale_out,
+                           int64_t R, int head_dim, int num_sms, int device, cudaStream_t stream);
+
 }  // namespace kq

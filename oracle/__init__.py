@@ -16,6 +16,10 @@ Parity status of each function (pins live in ``tests/test_oracle_pins.py``):
                     explicit Kronecker matrix.
   w4a4_gemm         pinned: brute-force integer loops on small inputs,
                     hand-derived extreme-code products, scale placement.
+  headwise_transform_quant
+                    pinned: equals the Kronecker path with P1 = I (one row
+                    per head), brute-force per-row quantisation, GQA head
+                    counts.
 """
 from __future__ import annotations
 
@@ -161,3 +165,24 @@ def w4a4_gemm(qx_packed, sx, qw_packed, sw) -> np.ndarray:
     qw = unpack_codes(qw_packed).astype(np.float64)
     acc = qx @ qw.T
     return acc * np.asarray(sx, dtype=np.float64)[:, None] * np.asarray(sw, dtype=np.float64)[None, :]
+
+
+def headwise_transform_quant(x_bits, Ph_bits, alpha: float, heads: int, head_dim: int,
+                             nthreads: Optional[int] = None):
+    """Per-head transform of the key / value cache (FlatQuant page: P_h and P_v
+    keep their full per-head shape; keys and values are transformed per head
+    and quantised before storage): every row x[t, h, :] of head_dim values is
+    multiplied by the same full factor Ph in fp64, then the INT4 rule of
+    ``quantize`` is applied to each (token, head) row on its own.
+
+    Returns dict(packed [T, heads*head_dim/2], scale32 [T, heads], scale64,
+    codes [T, heads*head_dim], dist) with rows (t, h) laid out as in x."""
+    x = np.asarray(x_bits, dtype=np.uint16).reshape(-1, heads * head_dim)
+    T = x.shape[0]
+    rows = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(T * heads, head_dim)
+    P = (np.asarray(Ph_bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    y = rows @ P.reshape(head_dim, head_dim)
+    r = quantize(y, alpha, nthreads)
+    return dict(packed=r["packed"].reshape(T, heads * head_dim // 2), scale32=r["scale32"].reshape(T, heads),
+                scale64=r["scale64"].reshape(T, heads), codes=r["codes"].reshape(T, heads * head_dim),
+                dist=r["dist"].reshape(T, heads * head_dim))

@@ -29,7 +29,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for must in ("kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_status_string",
-                 "kq_kernel_name", "kq_device_error", "kq_version", "kq_w4a4_gemm"):
+                 "kq_kernel_name", "kq_device_error", "kq_version", "kq_w4a4_gemm",
+                 "kq_headwise_transform_quant"):
         assert must in names
 
 
@@ -128,6 +129,25 @@ def test_w4a4_gemm_validation(kq):
     assert f(qx, sx, qw, sw, sw, 4, 8, 128, None) == kq.KQ_ERR_ARG        # y overlaps sw
     assert f(None, None, None, None, None, 0, 8, 128, None) == kq.KQ_OK   # empty: no-op
     assert f(None, None, None, None, None, 4, 0, 128, None) == kq.KQ_OK
+
+
+def test_headwise_validation(kq):
+    f = kq.lib.kq_headwise_transform_quant
+    x, P, q, s_ = 0x100000, 0x200000, 0x300000, 0x400000
+    assert f(x, P, 0.9, q, s_, -1, 8, 128, None) == kq.KQ_ERR_SHAPE
+    assert f(x, P, 0.9, q, s_, 4, 0, 128, None) == kq.KQ_ERR_SHAPE
+    assert f(x, P, 0.9, q, s_, 4, 8, 96, None) == kq.KQ_ERR_UNSUPPORTED
+    assert f(x, P, 0.9, q, s_, 4, 8, 256, None) == kq.KQ_ERR_UNSUPPORTED
+    assert f(x, P, 1.5, q, s_, 4, 8, 128, None) == kq.KQ_ERR_ARG
+    assert f(x, P, 0.0, q, s_, 4, 8, 128, None) == kq.KQ_ERR_ARG
+    assert f(x, P, 1e-7, q, s_, 4, 8, 128, None) == kq.KQ_ERR_UNSUPPORTED
+    assert f(x, None, 0.9, q, s_, 4, 8, 128, None) == kq.KQ_ERR_NULL
+    assert f(x + 2, P, 0.9, q, s_, 4, 8, 128, None) == kq.KQ_ERR_ALIGN
+    assert f(x, P, 0.9, q + 8, s_, 4, 8, 128, None) == kq.KQ_ERR_ALIGN
+    assert f(x, P, 0.9, x + 64, s_, 4, 8, 128, None) == kq.KQ_ERR_ARG   # codes over x
+    assert f(x, P, 0.9, q, q + 16, 4, 8, 128, None) == kq.KQ_ERR_ARG    # scales over codes
+    assert f(None, None, 0.9, None, None, 0, 8, 128, None) == kq.KQ_OK  # empty: no-op
+    assert f(x, P, 0.9, q, s_, 1 << 30, 8, 128, None) == kq.KQ_ERR_SHAPE
 
 
 def test_device_error_rejects_null(kq):
