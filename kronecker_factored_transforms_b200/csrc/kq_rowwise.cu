@@ -14,14 +14,15 @@
 // the fused transform kernel), D1 columns the rows of the slot.  One batch is 8
 // groups of H slots: stage 1 of the transform kernel with N = 128, A = Ph^T
 // (block-diagonal over the slots) resident in TMEM, B = the rows' x tile by TMA.
-// There is no second factor, so the epilogue reads D1 itself: per row (one D1
-// column) the absmax over the slot's lanes -- one warp reduction per column
-// and a shared-memory step across the warps of the slot -- then codes, 16-bit
-// stores into a swizzled staging tile and one TMA store per group.
+// There is no second factor, so the epilogue reads D1 itself, once: per row
+// (one D1 column) the absmax over the slot's lanes -- a local max, xor
+// shuffles within the warp and a shared-memory step across the warps of the
+// slot -- then codes, 16-bit stores into a swizzled staging tile and one TMA
+// store per group.
 //
 // Warps: 0 TMA producer | 1 TMEM allocator + MMA issuer | 4-7 and 8-11 two
-// epilogue warpgroups on alternate groups (4-7 and 8-11 also write Ph^T into
-// TMEM at start) | 2-3 idle.  Every mbarrier wait is bounded (kq_wait.cuh).
+// epilogue warpgroups on alternate batches (they also write Ph^T into TMEM at
+// start) | 2-3 idle.  Every mbarrier wait is bounded (kq_wait.cuh).
 #include <mutex>
 
 #include "kq_common.cuh"
@@ -54,15 +55,16 @@ struct RCfg {
     static constexpr int NB1 = (512 - A1COLS) / R1W; // 3
     static constexpr int RB = D / 2;                 // code bytes per row
     static constexpr int STG = H * RP * RB;          // staging bytes per group: 1 KB
-    static constexpr int OFF_STG = 0;                // 2 epilogues x 2 staging tiles
-    static constexpr int OFF_RAW = align_up_r(OFF_STG + 4 * STG, 1024);
-    static constexpr int SX = 6;                     // x tile stages
+    static constexpr int BSTG = GB * STG;            // per batch: 8 KB
+    static constexpr int OFF_STG = 0;                // 2 epilogues x 2 batch staging tiles
+    static constexpr int OFF_RAW = align_up_r(OFF_STG + 4 * BSTG, 1024);
+    static constexpr int SX = 5;                     // x tile stages
     static constexpr int FULL = 0, EMPTY = SX, D1FULL = 2 * SX, D1EMPTY = 2 * SX + NB1, TEARDOWN = 2 * SX + 2 * NB1;
     static constexpr int NBAR = TEARDOWN + 1;
     static constexpr int OFF_BAR = OFF_RAW + SX * XTILE;
     static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // TMEM base, abort flag, the constant 1, maxima
-    static constexpr int OFF_RED = OFF_MISC + 16;        // [2 epilogues][2 groups][4 warps][16] fp32
-    static constexpr int SMEM = OFF_RED + 2 * 2 * 4 * RP * 4 + 1024;
+    static constexpr int OFF_RED = OFF_MISC + 16;        // [2 epilogues][2 batches][GB][4 warps][16] fp32
+    static constexpr int SMEM = OFF_RED + 2 * 2 * GB * 4 * RP * 4 + 1024;
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     static_assert(STG % 1024 == 0 && OFF_RAW % 1024 == 0, "swizzle alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
@@ -104,7 +106,7 @@ __global__ void __launch_bounds__(R_THREADS, 1)
         }
         for (int b = 0; b < C::NB1; ++b) {
             mbar_init(bar(C::D1FULL + b), 1);
-            mbar_init(bar(C::D1EMPTY + b), C::GB * 4);  // each group's four epilogue warps
+            mbar_init(bar(C::D1EMPTY + b), 4);  // the four warps of the epilogue warpgroup
         }
         mbar_init(bar(C::TEARDOWN), 1);
         *s_abort = 0;
@@ -212,6 +214,9 @@ __global__ void __launch_bounds__(R_THREADS, 1)
         __syncwarp();
     } else if (warp >= 4 && warp < 12) {
         // ---------------- epilogue: per-row absmax, codes, staging, TMA store ----------------
+        // The two warpgroups take alternate batches (GB groups): a first pass over
+        // the groups finds the row maxima, one barrier, a second pass codes them;
+        // one TMA store writes the batch's rows.
         const int ew = (warp - 4) >> 2;
         const int q = warp & 3;
         const int et = tid - 128 - 128 * ew;
@@ -219,25 +224,24 @@ __global__ void __launch_bounds__(R_THREADS, 1)
         const int slot = (32 * q) / D;           // slot of this warp's lanes
         const int g8 = lane >> 2, qq = lane & 3;
         const int one = *reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
-        float *red = s_red + ew * 2 * 4 * RP;    // [2 buffers][4 warps][16 rows]
-        const uint32_t ng = uint32_t(nb) * C::GB;
-        const uint32_t stg0 = sbase + C::OFF_STG + 2 * ew * C::STG;
+        float *red = s_red + ew * (2 * C::GB * 4 * RP);  // [2 buffers][GB groups][4 warps][16 rows]
+        const uint32_t stg0 = sbase + C::OFF_STG + 2 * ew * C::BSTG;
         const bool storer = et == 0;
-        auto store_group = [&](int64_t gprev, int sb) {
+        auto store_batch = [&](int64_t gfirst, int sb) {
             if (storer) {
-                tma_store_2d(&tmap_q, 0, int(C::H * gprev * RP), stg0 + uint32_t(sb) * C::STG);
+                tma_store_2d(&tmap_q, 0, int(C::H * gfirst * RP), stg0 + uint32_t(sb) * C::BSTG);
                 bulk_commit();
             }
         };
         // this thread's two bytes of every row of its slot (see the transform kernel)
         const int row0 = slot * RP, bcol = ((32 * q) % D) / 2 + 2 * g8;
         const int swz_t = D == 128 ? qq : (qq >> 1);
-        int64_t g_prev = -1;
+        const int toff = (row0 + 2 * qq) * C::RB + ((((bcol >> 4) ^ swz_t) << 4) | (bcol & 15));
+        int64_t gprev = -1;
         int it = 0;
-        for (uint32_t gi = uint32_t(ew); gi < ng; gi += 2, ++it) {
-            const uint32_t jb = gi / C::GB, gp = gi % C::GB;
-            const uint32_t b = jb % C::NB1, ph = (jb / C::NB1) & 1u;
-            const int64_t g = (int64_t(blockIdx.x) + int64_t(jb) * gridDim.x) * C::GB + gp;
+        for (int64_t jb = ew; jb < nb; jb += 2, ++it) {
+            const uint32_t b = uint32_t(jb % C::NB1), ph = uint32_t((jb / C::NB1) & 1);
+            const int64_t g0 = (int64_t(blockIdx.x) + jb * gridDim.x) * C::GB;  // first group of the batch
             const int buf = it & 1;
             const bool ok = wait_bounded_err(bar(C::D1FULL + b), ph, s_abort, kSiteRowEpilogue, kWaitLimitNs,
                                              false, err);
@@ -245,65 +249,83 @@ __global__ void __launch_bounds__(R_THREADS, 1)
             if (named_barrier_any(nbar, 128, !warp_ok)) break;
             __syncwarp();
             tc_fence_after();
-            const uint32_t col = tmem + C::R1(int(b)) + uint32_t(RP * gp);
-            // per-row maxima over this warp's 32 lanes: one reduction per row
-            {
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(col + (uint32_t(32 * q) << 16), v);
+            const uint32_t colb = tmem + C::R1(int(b)) + (uint32_t(32 * q) << 16);
+            // pass 1: row maxima.  A 16x256b load per 16-lane half gives this thread
+            // lanes g8, g8 + 8 of both halves (four output columns) of rows
+            // 8 rep + 2 qq + d of each group; one x8 load covers four groups, so a
+            // batch takes two load rounds.  xor shuffles finish each row over the
+            // warp's lanes.
+#pragma unroll 1
+            for (int g4 = 0; g4 < C::GB; g4 += 4) {
+                uint32_t ra[32], rb[32];
+                tmem_ld_16x256b_x8(colb + uint32_t(RP * g4), ra);
+                tmem_ld_16x256b_x8(colb + (16u << 16) + uint32_t(RP * g4), rb);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < RP; ++i) {
-                    const uint32_t m = __reduce_max_sync(0xffffffffu, v[i] & 0x7FFFFFFFu);
-                    if (lane == i) red[(buf * 4 + q) * RP + i] = __uint_as_float(m);
+                for (int gl = 0; gl < 4; ++gl)
+#pragma unroll
+                    for (int rep = 0; rep < 2; ++rep)
+#pragma unroll
+                        for (int d = 0; d < 2; ++d) {
+                            const int o = 4 * (2 * gl + rep);
+                            float m = fmax3(fabsf(__uint_as_float(ra[o + d])), fabsf(__uint_as_float(ra[o + 2 + d])),
+                                            fabsf(__uint_as_float(rb[o + d])));
+                            m = fmaxf(m, fabsf(__uint_as_float(rb[o + 2 + d])));
+#pragma unroll
+                            for (int off = 4; off < 32; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+                            if (g8 == 0) red[((buf * C::GB + g4 + gl) * 4 + q) * RP + 8 * rep + 2 * qq + d] = m;
+                        }
+            }
+            if (storer) bulk_wait_read<0>();  // the store that read this staging tile is done
+            named_barrier_sync(nbar, 128);
+            if (gprev >= 0) store_batch(gprev, buf ^ 1);
+            unsigned char *stgb = smem + C::OFF_STG + (2 * ew + buf) * C::BSTG + toff;
+            // pass 2: scales and codes, four groups per load round
+#pragma unroll 1
+            for (int g4 = 0; g4 < C::GB; g4 += 4) {
+                uint32_t ra[32], rb[32];
+                tmem_ld_16x256b_x8(colb + uint32_t(RP * g4), ra);
+                tmem_ld_16x256b_x8(colb + (16u << 16) + uint32_t(RP * g4), rb);
+                tmem_wait_ld();
+                if (g4 + 4 >= C::GB) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(C::D1EMPTY + b));  // this warp is done with the region
+                }
+#pragma unroll
+                for (int gl = 0; gl < 4; ++gl) {
+                    const int gp = g4 + gl;
+                    unsigned char *tbase = stgb + gp * C::STG;
+#pragma unroll
+                    for (int rep = 0; rep < 2; ++rep)
+#pragma unroll
+                        for (int d = 0; d < 2; ++d) {
+                            const int i = 8 * rep + 2 * qq + d;
+                            float m = 0.0f;
+#pragma unroll
+                            for (int w = 0; w < 4; ++w)
+                                if ((32 * w) / D == slot) m = fmaxf(m, red[((buf * C::GB + gp) * 4 + w) * RP + i]);
+                            const float sc = alpha * m * (1.0f / 7.0f);
+                            const float iv = sc > 0.0f ? fminf(__fdividef(1.0f, sc), 3.0e38f) : 0.0f;
+                            // the scale of row i of the slot: written once, by the slot's first warp
+                            if ((32 * q) % D == 0 && g8 == 0) {
+                                const int64_t r = (C::H * (g0 + gp) + slot) * RP + i;
+                                if (r < R) scale_out[r] = sc;
+                            }
+                            const int o = 4 * (2 * gl + rep);
+                            const uint32_t wb = pack_s4x2(round_code_r(rb[o + 2 + d], iv, one),
+                                                          round_code_r(rb[o + d], iv, one), 0u);
+                            const uint32_t w = pack_s4x2(round_code_r(ra[o + 2 + d], iv, one),
+                                                         round_code_r(ra[o + d], iv, one), wb);
+                            *reinterpret_cast<uint16_t *>(tbase + (8 * rep + d) * C::RB) = uint16_t(w);
+                        }
                 }
             }
-            if (storer) bulk_wait_read<0>();
-            named_barrier_sync(nbar, 128);
-            if (g_prev >= 0) store_group(g_prev, buf ^ 1);
-            // scales of the four rows this thread codes: 2 qq, 2 qq + 1, 8 + 2 qq, 9 + 2 qq
-            float inv[2][2];
-#pragma unroll
-            for (int rep = 0; rep < 2; ++rep)
-#pragma unroll
-                for (int d = 0; d < 2; ++d) {
-                    const int i = 8 * rep + 2 * qq + d;
-                    float m = 0.0f;
-#pragma unroll
-                    for (int w = 0; w < 4; ++w)
-                        if ((32 * w) / D == slot) m = fmaxf(m, red[(buf * 4 + w) * RP + i]);
-                    const float s = alpha * m * (1.0f / 7.0f);
-                    inv[rep][d] = s > 0.0f ? fminf(__fdividef(1.0f, s), 3.0e38f) : 0.0f;
-                    // the scale of row i of the slot: written once, by the slot's first warp
-                    if ((32 * q) % D == 0 && g8 == 0) {
-                        const int64_t r = (C::H * g + slot) * RP + i;
-                        if (r < R) scale_out[r] = s;
-                    }
-                }
-            unsigned char *stg = smem + C::OFF_STG + (2 * ew + buf) * C::STG;
-            unsigned char *tbase = stg + (row0 + 2 * qq) * C::RB + ((((bcol >> 4) ^ swz_t) << 4) | (bcol & 15));
-            uint32_t ra[8], rb[8];
-            tmem_ld_16x256b_x2(col + (uint32_t(32 * q) << 16), ra);
-            tmem_ld_16x256b_x2(col + (uint32_t(32 * q + 16) << 16), rb);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::D1EMPTY + b));  // this warp is done reading the group
-#pragma unroll
-            for (int rep = 0; rep < 2; ++rep)
-#pragma unroll
-                for (int d = 0; d < 2; ++d) {
-                    const float iv = inv[rep][d];
-                    const uint32_t wb = pack_s4x2(round_code_r(rb[4 * rep + 2 + d], iv, one),
-                                                  round_code_r(rb[4 * rep + d], iv, one), 0u);
-                    const uint32_t w = pack_s4x2(round_code_r(ra[4 * rep + 2 + d], iv, one),
-                                                 round_code_r(ra[4 * rep + d], iv, one), wb);
-                    *reinterpret_cast<uint16_t *>(tbase + (8 * rep + d) * C::RB) = uint16_t(w);
-                }
             fence_proxy_async_smem();
-            g_prev = g;
+            gprev = g0;
         }
         named_barrier_sync(nbar, 128);
-        if (g_prev >= 0) store_group(g_prev, (it - 1) & 1);
+        if (gprev >= 0) store_batch(gprev, (it - 1) & 1);
         if (storer) bulk_wait<0>();
     }
 
@@ -344,7 +366,7 @@ cudaError_t launch_rowwise_inst(const uint16_t *x, const uint16_t *Ph, float alp
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     const cuuint64_t dq[2] = {cuuint64_t(C::RB), cuuint64_t(R)};
     const cuuint64_t sq[1] = {cuuint64_t(C::RB)};
-    const cuuint32_t bq[2] = {cuuint32_t(C::RB), cuuint32_t(C::H * RP)};
+    const cuuint32_t bq[2] = {cuuint32_t(C::RB), cuuint32_t(C::GB * C::H * RP)};  // one batch
     r = encode(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q_out, dq, sq, bq, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
