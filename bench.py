@@ -43,7 +43,9 @@ PROFILES = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = ["kronecker_factored_transforms_b200/csrc/kq_tc05.cu",
                   "kronecker_factored_transforms_b200/csrc/kq_tc05_ptx.cuh",
                   "kronecker_factored_transforms_b200/csrc/kq_warp_mma.cu",
-                  "kronecker_factored_transforms_b200/csrc/kq_common.cuh"]
+                  "kronecker_factored_transforms_b200/csrc/kq_common.cuh",
+                  "kronecker_factored_transforms_b200/csrc/kq_tile.cuh",
+                  "kronecker_factored_transforms_b200/csrc/kq_wait.cuh"]
 
 
 def parse():
@@ -52,9 +54,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["transform", "gemm"], default="transform",
+    ap.add_argument("--workload", choices=["transform", "gemm", "two_stage"], default="transform",
                     help="transform: the fused transform + INT4 path (default); gemm: the W4A4 product "
-                         "of packed codes that consumes it (M = N = K = 8192)")
+                         "of packed codes that consumes it (M = N = K = 8192); two_stage: the path for "
+                         "factors above 128 (--two-stage-config)")
+    ap.add_argument("--two-stage-config", choices=["square65536", "ffn28672"], default="square65536")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0,
@@ -283,12 +287,82 @@ def run_gemm(args):
     return 0
 
 
+def run_two_stage(args):
+    """The two-stage path for factors above 128 on one large-factor workload.
+    One step is one kq_transform_quant_two_stage call (stage 1 and stage 2
+    kernels); x and the outputs rotate over two buffer sets, and the 4 T n
+    byte workspace is rewritten every step.  Roofline: the slower of the
+    algorithmic bytes (2.5 n + 4 per token) at the measured HBM peak and the
+    factored flops 2 n (n1 + n2) per token at the measured bf16 peak.
+    Single GPU only."""
+    import torch
+    from kronecker_factored_transforms_b200 import _lib
+    name = args.two_stage_config
+    w = make_workload(name)
+    T, n1, n2, n = w.T, w.n1, w.n2, w.n
+    dev = torch.device("cuda", 0)
+    R = 2
+    xs = [torch.from_numpy(w.x.view(np.int16)).to(dev) for _ in range(R)]
+    qs = [torch.empty((T, n // 2), dtype=torch.uint8, device=dev) for _ in range(R)]
+    ss = [torch.empty((T,), dtype=torch.float32, device=dev) for _ in range(R)]
+    need = _lib.kq_two_stage_workspace_bytes(T, n1, n2)
+    ws = torch.empty((need,), dtype=torch.uint8, device=dev)
+    P1 = torch.from_numpy(w.P1.view(np.int16)).to(dev)
+    P2 = torch.from_numpy(w.P2.view(np.int16)).to(dev)
+    cinv = torch.from_numpy(w.cinv).to(dev) if w.cinv is not None else None
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        _lib.kq_transform_quant_two_stage(xs[i % R], P1, P2, cinv, w.alpha, qs[i % R], ss[i % R], ws, need,
+                                          T, n1, n2, stream=stream.cuda_stream)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(0)
+    with sampler:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    if _lib.kq_device_error(stream) != 0:
+        raise RuntimeError("a bounded wait timed out inside the kernel")
+    ms = e0.elapsed_time(e1) / args.steps
+    hbm_peak, tf_peak, kind = measured_peaks()
+    bytes_launch, flops_launch = workload_bytes(T, n), workload_flops(T, n1, n2)
+    t_hbm, t_tc = bytes_launch / (hbm_peak * 1e9), flops_launch / (tf_peak * 1e12)
+    sec = ms / 1e3
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": bytes_launch / sec / 1e9, "peak": hbm_peak, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops_launch / sec / 1e12, "peak": tf_peak, "unit": "TFLOP/s"}
+    roof.update({"frac": roof["achieved"] / roof["peak"], "traffic": None,
+                 "peak_source": "%s (MEASURED_PEAKS.json)" % kind, "bytes_per_launch": bytes_launch,
+                 "flops_per_launch": flops_launch, "roofline_time_us": 1e6 * max(t_hbm, t_tc),
+                 "measured_time_us": 1e3 * ms, "workspace_bytes": need})
+    line = {"metric": "tokens/s and % roofline of the two-stage Kronecker transform+INT4 (factors above 128)",
+            "value": T / sec, "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "%s: T=%d, n=%d (n1=%d, n2=%d), alpha=%g, cinv %s" % (
+                name, T, n, n1, n2, w.alpha, "per channel" if w.cinv is not None else "none"),
+                       "T": T, "n1": n1, "n2": n2, "l2": "x and outputs rotate over 2 sets; the workspace "
+                                                          "(%d MB) is rewritten every step" % (need >> 20)},
+            "roofline": roof, "gpu_launches": 2 * args.steps, "clocks": sampler.report()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.workload == "gemm":
         return run_gemm(args)
+    if args.workload == "two_stage":
+        return run_two_stage(args)
 
     import torch
     import torch.distributed as dist

@@ -154,6 +154,38 @@ kq_status kq_headwise_transform_quant(const uint16_t *x, const uint16_t *Ph, flo
                                       float *scale_out, int64_t T, int heads, int head_dim, kq_stream_t stream);
 
 /*
+ * kq_transform_quant_two_stage -- kq_transform_quant for factors up to 256
+ * (FlatQuant page, "The fused kernel", Figure 8 (c): factors too large for one
+ * on-chip pass; the transform runs as two stages with the intermediate in
+ * global memory).  Same result and INT4 rule as kq_transform_quant:
+ * Y~ = P1^T X~ P2 for the row-major n1 x n2 view X~ of x o cinv, per-token
+ * s = alpha * max|y| / 7, codes clamp(round_half_even(y / s), -8, 7), two per
+ * byte with element 2k in the low nibble, output element k = i * n2 + j.
+ * Stage 1 writes Z^T = (X~ P2)^T of every token to `workspace` as a hi/lo
+ * bf16 pair; stage 2 forms P1^T Z per token, quantises and packs.  Neither
+ * Y~ nor an fp32 intermediate reaches global memory.
+ *
+ * x, P1, P2, cinv, alpha, q_out, scale_out, T, n1, n2: as kq_transform_quant,
+ *           except that n1 and n2 are multiples of 16 in [16, 256] and
+ *           T * n1 * n2 < 2^31.
+ * workspace caller-owned device scratch of at least
+ *           kq_two_stage_workspace_bytes(T, n1, n2) = 4 * T * n1 * n2 bytes,
+ *           16-byte aligned; overwritten, and must stay untouched until the
+ *           work on `stream` has finished.
+ * Returns KQ_ERR_SHAPE, KQ_ERR_UNSUPPORTED (factor size, or alpha below
+ * 2^-19), KQ_ERR_ARG (alpha outside (0, 1], workspace too small, overlapping
+ * buffers), KQ_ERR_NULL, KQ_ERR_ALIGN, KQ_ERR_CUDA.  Asynchronous on
+ * `stream`; allocates nothing.
+ */
+kq_status kq_transform_quant_two_stage(const uint16_t *x, const uint16_t *P1, const uint16_t *P2,
+                                       const float *cinv, float alpha, uint8_t *q_out, float *scale_out,
+                                       void *workspace, uint64_t workspace_bytes, int64_t T, int n1, int n2,
+                                       kq_stream_t stream);
+
+/* Workspace bytes kq_transform_quant_two_stage needs: 4 * T * n1 * n2 (0 for T <= 0). */
+uint64_t kq_two_stage_workspace_bytes(int64_t T, int n1, int n2);
+
+/*
  * kq_device_error -- read and clear the device-side status word that the
  * kernels set when a bounded wait gives up (they then skip their remaining
  * work instead of hanging).  Synchronises `stream`.  *code receives 0 when

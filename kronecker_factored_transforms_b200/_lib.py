@@ -43,9 +43,13 @@ def _load() -> ctypes.CDLL:
     lib.kq_selftest_bounded_wait.argtypes = [I64, P]
     lib.kq_w4a4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P]
     lib.kq_headwise_transform_quant.argtypes = [P, P, F32, P, P, I64, I32, I32, P]
+    lib.kq_transform_quant_two_stage.argtypes = [P, P, P, P, F32, P, P, P, ctypes.c_uint64, I64, I32, I32, P]
     for f in (lib.kq_transform_quant, lib.kq_transform, lib.kq_dequant_inverse, lib.kq_device_error,
-              lib.kq_selftest_bounded_wait, lib.kq_w4a4_gemm, lib.kq_headwise_transform_quant):
+              lib.kq_selftest_bounded_wait, lib.kq_w4a4_gemm, lib.kq_headwise_transform_quant,
+              lib.kq_transform_quant_two_stage):
         f.restype = ctypes.c_int
+    lib.kq_two_stage_workspace_bytes.argtypes = [I64, I32, I32]
+    lib.kq_two_stage_workspace_bytes.restype = ctypes.c_uint64
     lib.kq_status_string.argtypes = [I32]
     lib.kq_status_string.restype = ctypes.c_char_p
     lib.kq_kernel_name.argtypes = [I32, I32, I32]
@@ -59,7 +63,7 @@ lib = _load()
 
 EXPORTED = ("kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_device_error",
             "kq_selftest_bounded_wait", "kq_status_string", "kq_kernel_name", "kq_version", "kq_w4a4_gemm",
-            "kq_headwise_transform_quant")
+            "kq_headwise_transform_quant", "kq_transform_quant_two_stage", "kq_two_stage_workspace_bytes")
 
 
 def _ptr(t) -> Optional[int]:
@@ -97,6 +101,18 @@ def kq_headwise_transform_quant(x, Ph, alpha: float, q_out, scale_out, T: int, h
     _check("kq_headwise_transform_quant",
            lib.kq_headwise_transform_quant(_ptr(x), _ptr(Ph), float(alpha), _ptr(q_out), _ptr(scale_out), int(T),
                                            int(heads), int(head_dim), _stream(stream)))
+
+
+def kq_two_stage_workspace_bytes(T: int, n1: int, n2: int) -> int:
+    return int(lib.kq_two_stage_workspace_bytes(int(T), int(n1), int(n2)))
+
+
+def kq_transform_quant_two_stage(x, P1, P2, cinv, alpha: float, q_out, scale_out, workspace, workspace_bytes: int,
+                                 T: int, n1: int, n2: int, stream=None) -> None:
+    _check("kq_transform_quant_two_stage",
+           lib.kq_transform_quant_two_stage(_ptr(x), _ptr(P1), _ptr(P2), _ptr(cinv), float(alpha), _ptr(q_out),
+                                            _ptr(scale_out), _ptr(workspace), int(workspace_bytes), int(T), int(n1),
+                                            int(n2), _stream(stream)))
 
 
 def kq_w4a4_gemm(qx, sx, qw, sw, y, M: int, N: int, K: int, stream=None) -> None:

@@ -206,6 +206,57 @@ kq_status kq_headwise_transform_quant(const uint16_t *x, const uint16_t *Ph, flo
     return err == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;
 }
 
+kq_status kq_transform_quant_two_stage(const uint16_t *x, const uint16_t *P1, const uint16_t *P2,
+                                       const float *cinv, float alpha, uint8_t *q_out, float *scale_out,
+                                       void *workspace, uint64_t workspace_bytes, int64_t T, int n1, int n2,
+                                       kq_stream_t stream) {
+    if (T < 0 || n1 <= 0 || n2 <= 0) return KQ_ERR_SHAPE;
+    if (!kq::two_stage_supports(n1, n2)) return KQ_ERR_UNSUPPORTED;
+    const int64_t n = int64_t(n1) * n2;
+    if (T >= (int64_t(1) << 31) / n) return KQ_ERR_SHAPE;  // rows and offsets are 32-bit
+    kq_status st = check_alpha(alpha);
+    if (st != KQ_OK) return st;
+    if (!(alpha >= 0x1p-19f)) return KQ_ERR_UNSUPPORTED;  // the code rounding's range
+    if (T == 0) return KQ_OK;
+    if (!x || !P1 || !P2 || !q_out || !scale_out || !workspace) return KQ_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(P1, 16) || !aligned(P2, 16) || !aligned(q_out, 16) ||
+        !aligned(workspace, 16) || !aligned(scale_out, 4) || (cinv && !aligned(cinv, 16)))
+        return KQ_ERR_ALIGN;
+    const uint64_t need = kq::two_stage_workspace_bytes(T, n1, n2);
+    if (workspace_bytes < need) return KQ_ERR_ARG;
+    const Range in[4] = {range_of(x, uint64_t(T) * n * 2), range_of(P1, uint64_t(n1) * n1 * 2),
+                         range_of(P2, uint64_t(n2) * n2 * 2), range_of(cinv, cinv ? uint64_t(n) * 4 : 0)};
+    const Range out[3] = {range_of(q_out, uint64_t(T) * n / 2), range_of(scale_out, uint64_t(T) * 4),
+                          range_of(workspace, need)};
+    for (const Range &o : out)
+        for (const Range &i : in)
+            if (overlap(o, i)) return KQ_ERR_ARG;
+    if (overlap(out[0], out[1]) || overlap(out[0], out[2]) || overlap(out[1], out[2])) return KQ_ERR_ARG;
+    DeviceInfo info;
+    if ((st = device_info(info)) != KQ_OK) return st;
+    kq::LaunchArgs a;
+    a.x = x;
+    a.P1 = P1;
+    a.P2 = P2;
+    a.cinv = cinv;
+    a.alpha = alpha;
+    a.q_out = q_out;
+    a.scale_out = scale_out;
+    a.y_out = nullptr;
+    a.T = T;
+    a.n1 = n1;
+    a.n2 = n2;
+    a.num_sms = info.num_sms;
+    a.device = info.device;
+    a.stream = reinterpret_cast<cudaStream_t>(stream);
+    return kq::launch_two_stage(a, workspace) == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;
+}
+
+uint64_t kq_two_stage_workspace_bytes(int64_t T, int n1, int n2) {
+    if (T <= 0 || n1 <= 0 || n2 <= 0) return 0;
+    return kq::two_stage_workspace_bytes(T, n1, n2);
+}
+
 kq_status kq_device_error(kq_stream_t stream, int *code) {
     if (!code) return KQ_ERR_NULL;
     unsigned int v = 0;

@@ -56,4 +56,10 @@ cudaError_t launch_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *
 cudaError_t launch_rowwise(const uint16_t *x, const uint16_t *Ph, float alpha, uint8_t *q_out, float *scale_out,
                            int64_t R, int head_dim, int num_sms, int device, cudaStream_t stream);
 
+// Two-stage transform + INT4 for factors up to 256 through a workspace of
+// two_stage_workspace_bytes(T, n1, n2) bytes (Z^T hi then lo, bf16).
+bool two_stage_supports(int n1, int n2);
+uint64_t two_stage_workspace_bytes(int64_t T, int n1, int n2);
+cudaError_t launch_two_stage(const LaunchArgs &a, void *workspace);
+
 }  // namespace kq

@@ -122,6 +122,15 @@ CONFIGS = {
     "sweep4096": dict(T=1024, n1=64, n2=64, seed=4, alpha=0.9, factors="orthogonal",
                       x_kind="normal", outliers=("frac", 0.01, 30.0), pivot=None,
                       scaled=False),
+    # Factors above 128 (the two-stage path).  n=28672 (112x256), the FFN width
+    # of a 70B-class model; the mlp14336 recipe otherwise; seed 5.
+    "ffn28672": dict(T=2048, n1=112, n2=256, seed=5, alpha=0.9, factors="orthogonal",
+                     x_kind="relu_gated", outliers=("frac", 0.005, 40.0), pivot=None,
+                     scaled=False),
+    # n=65536 (256x256), both factors above 128; the hidden8192 recipe
+    # otherwise (Student-t, c ~ logU[0.5, 2], near-identity factors); seed 6.
+    "square65536": dict(T=1024, n1=256, n2=256, seed=6, alpha=0.85, factors="near_identity",
+                        x_kind="student_t", outliers=None, pivot=None, scaled=True),
 }
 
 SWEEP_T = (1, 16, 128, 1024, 16384, 65536)

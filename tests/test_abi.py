@@ -30,7 +30,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for must in ("kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_status_string",
                  "kq_kernel_name", "kq_device_error", "kq_version", "kq_w4a4_gemm",
-                 "kq_headwise_transform_quant"):
+                 "kq_headwise_transform_quant", "kq_transform_quant_two_stage", "kq_two_stage_workspace_bytes"):
         assert must in names
 
 
@@ -148,6 +148,31 @@ def test_headwise_validation(kq):
     assert f(x, P, 0.9, q, q + 16, 4, 8, 128, None) == kq.KQ_ERR_ARG    # scales over codes
     assert f(None, None, 0.9, None, None, 0, 8, 128, None) == kq.KQ_OK  # empty: no-op
     assert f(x, P, 0.9, q, s_, 1 << 30, 8, 128, None) == kq.KQ_ERR_SHAPE
+
+
+def test_two_stage_validation(kq):
+    f = kq.lib.kq_transform_quant_two_stage
+    x, P1, P2, c, q, s_, w = 0x1000000, 0x2000000, 0x3000000, 0x4000000, 0x5000000, 0x6000000, 0x10000000
+    T, n1, n2 = 4, 256, 256
+    need = kq.kq_two_stage_workspace_bytes(T, n1, n2)
+    assert need == 4 * T * n1 * n2
+    assert kq.kq_two_stage_workspace_bytes(0, 256, 256) == 0 and kq.kq_two_stage_workspace_bytes(-3, 16, 16) == 0
+    ok = (x, P1, P2, c, 0.9, q, s_, w, need)
+    assert f(*ok[:8], need, -1, n1, n2, None) == kq.KQ_ERR_SHAPE
+    assert f(*ok[:8], need, T, 0, n2, None) == kq.KQ_ERR_SHAPE
+    for bad in ((272, 256), (256, 24), (8, 64), (64, 512)):
+        assert f(*ok[:8], need, T, bad[0], bad[1], None) == kq.KQ_ERR_UNSUPPORTED
+    assert f(*ok[:8], need, 1 << 15, 256, 256, None) == kq.KQ_ERR_SHAPE      # T n = 2^31
+    assert f(x, P1, P2, c, 1.5, q, s_, w, need, T, n1, n2, None) == kq.KQ_ERR_ARG
+    assert f(x, P1, P2, c, 1e-7, q, s_, w, need, T, n1, n2, None) == kq.KQ_ERR_UNSUPPORTED
+    assert f(*ok[:8], need - 1, T, n1, n2, None) == kq.KQ_ERR_ARG            # workspace too small
+    assert f(x, P1, P2, c, 0.9, q, s_, None, need, T, n1, n2, None) == kq.KQ_ERR_NULL
+    assert f(x, P1, P2, c, 0.9, q, s_, w + 8, need, T, n1, n2, None) == kq.KQ_ERR_ALIGN
+    assert f(x, P1, P2, c + 4, 0.9, q, s_, w, need, T, n1, n2, None) == kq.KQ_ERR_ALIGN
+    assert f(x, P1, P2, c, 0.9, q, s_, x + 1024, need, T, n1, n2, None) == kq.KQ_ERR_ARG   # workspace over x
+    assert f(x, P1, P2, c, 0.9, q, s_, q + 16, need, T, n1, n2, None) == kq.KQ_ERR_ARG     # workspace over codes
+    assert f(x, P1, P2, c, 0.9, q, q + 64, w, need, T, n1, n2, None) == kq.KQ_ERR_ARG      # scales over codes
+    assert f(None, None, None, None, 0.9, None, None, None, 0, 0, n1, n2, None) == kq.KQ_OK  # empty: no-op
 
 
 def test_device_error_rejects_null(kq):
