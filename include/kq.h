@@ -182,6 +182,32 @@ kq_status kq_transform_quant_two_stage(const uint16_t *x, const uint16_t *P1, co
                                        void *workspace, uint64_t workspace_bytes, int64_t T, int n1, int n2,
                                        kq_stream_t stream);
 
+/*
+ * kq_transform_quant_two_stage_static -- kq_transform_quant_two_stage with
+ * its workspace taken from a static device array inside libkq instead of a
+ * caller buffer, so the call allocates nothing and needs no scratch from the
+ * caller.  The pages have no counterpart for this entry: it is a convenience
+ * of this library for callers without an allocator at hand.
+ *
+ * Arguments and results as kq_transform_quant_two_stage (without workspace
+ * and workspace_bytes).  Limit: 4 * T * n1 * n2 <= KQ_STATIC_WORKSPACE_BYTES
+ * (64 MiB: e.g. T <= 256 at n1 = n2 = 256); a larger request returns
+ * KQ_ERR_ARG before anything is launched.
+ *
+ * The array is ONE per device and process, shared by every call of this entry
+ * on that device.  Two calls whose work can overlap on the device -- issued on
+ * different streams without an ordering between them, or from several host
+ * threads -- race on it and can return wrong codes; calls on one stream are
+ * ordered and safe.  The first call on a device looks up the array's address
+ * (cudaGetSymbolAddress, which can load the module) and must come before any
+ * stream capture on that device.  Nothing is claimed about calling this entry
+ * inside a captured graph.
+ */
+#define KQ_STATIC_WORKSPACE_BYTES (64ull * 1024ull * 1024ull)
+kq_status kq_transform_quant_two_stage_static(const uint16_t *x, const uint16_t *P1, const uint16_t *P2,
+                                              const float *cinv, float alpha, uint8_t *q_out, float *scale_out,
+                                              int64_t T, int n1, int n2, kq_stream_t stream);
+
 /* Workspace bytes kq_transform_quant_two_stage needs: 4 * T * n1 * n2 (0 for T <= 0). */
 uint64_t kq_two_stage_workspace_bytes(int64_t T, int n1, int n2);
 

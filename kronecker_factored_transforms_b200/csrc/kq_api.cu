@@ -257,6 +257,24 @@ uint64_t kq_two_stage_workspace_bytes(int64_t T, int n1, int n2) {
     return kq::two_stage_workspace_bytes(T, n1, n2);
 }
 
+kq_status kq_transform_quant_two_stage_static(const uint16_t *x, const uint16_t *P1, const uint16_t *P2,
+                                              const float *cinv, float alpha, uint8_t *q_out, float *scale_out,
+                                              int64_t T, int n1, int n2, kq_stream_t stream) {
+    static_assert(KQ_STATIC_WORKSPACE_BYTES == kq::kStaticScratchBytes, "static workspace size");
+    if (T < 0 || n1 <= 0 || n2 <= 0) return KQ_ERR_SHAPE;
+    if (!kq::two_stage_supports(n1, n2)) return KQ_ERR_UNSUPPORTED;
+    if (T > int64_t(kq::kStaticScratchBytes / (uint64_t(4) * uint64_t(n1) * uint64_t(n2)))) return KQ_ERR_ARG;
+    void *scratch = nullptr;
+    if (T > 0) {
+        DeviceInfo info;
+        kq_status st = device_info(info);
+        if (st != KQ_OK) return st;
+        if (kq::static_scratch(info.device, &scratch) != cudaSuccess) return KQ_ERR_CUDA;
+    }
+    return kq_transform_quant_two_stage(x, P1, P2, cinv, alpha, q_out, scale_out, scratch, kq::kStaticScratchBytes, T,
+                                        n1, n2, stream);
+}
+
 kq_status kq_device_error(kq_stream_t stream, int *code) {
     if (!code) return KQ_ERR_NULL;
     unsigned int v = 0;

@@ -62,4 +62,8 @@ bool two_stage_supports(int n1, int n2);
 uint64_t two_stage_workspace_bytes(int64_t T, int n1, int n2);
 cudaError_t launch_two_stage(const LaunchArgs &a, void *workspace);
 
+// The static workspace of kq_transform_quant_two_stage_static (one per device).
+constexpr uint64_t kStaticScratchBytes = uint64_t(64) << 20;
+cudaError_t static_scratch(int device, void **ptr);
+
 }  // namespace kq
