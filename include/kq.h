@@ -169,9 +169,10 @@ kq_status kq_headwise_transform_quant(const uint16_t *x, const uint16_t *Ph, flo
  *           except that n1 and n2 are multiples of 16 in [16, 256] and
  *           T * n1 * n2 < 2^31.
  * workspace caller-owned device scratch of at least
- *           kq_two_stage_workspace_bytes(T, n1, n2) = 4 * T * n1 * n2 bytes,
- *           16-byte aligned; overwritten, and must stay untouched until the
- *           work on `stream` has finished.
+ *           kq_two_stage_workspace_bytes(T, n1, n2) = 4 * T * n1 * Jp bytes,
+ *           Jp = 128 * ceil(n2 / 128) (Z^T rows per token, padded to whole
+ *           128-row slices), 16-byte aligned; overwritten, and must stay
+ *           untouched until the work on `stream` has finished.
  * Returns KQ_ERR_SHAPE, KQ_ERR_UNSUPPORTED (factor size, or alpha below
  * 2^-19), KQ_ERR_ARG (alpha outside (0, 1], workspace too small, overlapping
  * buffers), KQ_ERR_NULL, KQ_ERR_ALIGN, KQ_ERR_CUDA.  Asynchronous on
@@ -190,9 +191,9 @@ kq_status kq_transform_quant_two_stage(const uint16_t *x, const uint16_t *P1, co
  * of this library for callers without an allocator at hand.
  *
  * Arguments and results as kq_transform_quant_two_stage (without workspace
- * and workspace_bytes).  Limit: 4 * T * n1 * n2 <= KQ_STATIC_WORKSPACE_BYTES
- * (64 MiB: e.g. T <= 256 at n1 = n2 = 256); a larger request returns
- * KQ_ERR_ARG before anything is launched.
+ * and workspace_bytes).  Limit: kq_two_stage_workspace_bytes(T, n1, n2) <=
+ * KQ_STATIC_WORKSPACE_BYTES (64 MiB: e.g. T <= 256 at n1 = n2 = 256); a larger
+ * request returns KQ_ERR_ARG before anything is launched.
  *
  * The array is ONE per device and process, shared by every call of this entry
  * on that device.  Two calls whose work can overlap on the device -- issued on
@@ -208,7 +209,7 @@ kq_status kq_transform_quant_two_stage_static(const uint16_t *x, const uint16_t 
                                               const float *cinv, float alpha, uint8_t *q_out, float *scale_out,
                                               int64_t T, int n1, int n2, kq_stream_t stream);
 
-/* Workspace bytes kq_transform_quant_two_stage needs: 4 * T * n1 * n2 (0 for T <= 0). */
+/* Workspace bytes kq_transform_quant_two_stage needs: 4 * T * n1 * 128 * ceil(n2 / 128) (0 for T <= 0). */
 uint64_t kq_two_stage_workspace_bytes(int64_t T, int n1, int n2);
 
 /*

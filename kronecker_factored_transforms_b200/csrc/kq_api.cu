@@ -263,7 +263,7 @@ kq_status kq_transform_quant_two_stage_static(const uint16_t *x, const uint16_t 
     static_assert(KQ_STATIC_WORKSPACE_BYTES == kq::kStaticScratchBytes, "static workspace size");
     if (T < 0 || n1 <= 0 || n2 <= 0) return KQ_ERR_SHAPE;
     if (!kq::two_stage_supports(n1, n2)) return KQ_ERR_UNSUPPORTED;
-    if (T > int64_t(kq::kStaticScratchBytes / (uint64_t(4) * uint64_t(n1) * uint64_t(n2)))) return KQ_ERR_ARG;
+    if (T > int64_t(kq::kStaticScratchBytes / kq::two_stage_workspace_bytes(1, n1, n2))) return KQ_ERR_ARG;
     void *scratch = nullptr;
     if (T > 0) {
         DeviceInfo info;

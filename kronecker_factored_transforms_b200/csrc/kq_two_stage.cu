@@ -11,24 +11,26 @@
 //
 // The intermediate leaves stage 1 as a hi/lo bf16 pair (Z = hi + lo, about 16
 // significant bits, the same split the fused kernel applies on chip) in a
-// caller-provided workspace of 4 T n bytes: hi [T][n2][n1] then lo [T][n2][n1].
-// One token's whole Y~ (n / 128 TMEM columns, at most 512) stays in TMEM until
-// its absmax is known, so the codes leave from the stage-2 kernel and neither
-// Y~ nor an fp32 intermediate is ever written.  Factors are multiples of 16 up
-// to 256 (n up to 65536).
+// caller-provided workspace: hi [T][Jp][n1] then lo [T][Jp][n1] with
+// Jp = 128 ceil(n2 / 128) rows per token (rows j >= n2 hold zeros).  One
+// token's whole Y~ (at most 512 TMEM columns) stays in TMEM until its absmax
+// is known, so the codes leave from the stage-2 kernel and neither Y~ nor an
+// fp32 intermediate is ever written.  Factors are multiples of 16 up to 256.
 //
-// Stage 1 (512 threads, one 128-wide slice of j per CTA, persistent over row
-// tiles of 128 rows (t, a)): warp 0 TMA loads of x tiles [128 rows] x [64 b];
-// warp 1 TMEM allocation and MMA issue (A = the slice of P2^T, resident in
-// TMEM; B = the x' hi and lo tiles; N = 128); warps 4-11 split x o cinv into
-// hi/lo tiles (without cinv the MMA reads the loaded tile as is); warps 12-15
-// write P2^T into TMEM, then split each accumulator tile into Z^T hi/lo and
-// store it.
+// Stage 1 (512 threads, persistent over tiles of 64 rows (t, a)): warp 0 TMA
+// loads of x tiles [64 rows] x [64 b]; warp 1 TMEM allocation and MMA issue
+// (A = P2^T in 128-row slices of j, resident in TMEM; B = the x' hi and lo
+// tiles; N = 64); warps 4-11 split x o cinv into hi/lo tiles, with cinv loaded
+// one chunk ahead (without cinv the MMA reads the loaded tile as is); warps
+// 12-15 write P2^T into TMEM, then split each accumulator into Z^T hi/lo and
+// store it with TMA tensor stores of [128 j] x [16 a] boxes.
 //
 // Stage 2 (384 threads, persistent over tokens): warp 0 TMA loads of Z^T hi/lo
 // tiles [128 j] x [64 a]; warp 1 TMEM allocation and MMA issue (A = the Z^T
-// tiles, B = P1^T resident in shared memory, N = n1); warps 4-11 the epilogue
-// (two warpgroups, each half of every 128-lane block's columns).
+// tiles, B = P1^T resident in shared memory, N = n1), one 128-lane slice of j
+// at a time; warps 4-11 the epilogue (two warpgroups, each half of every
+// slice's columns).  Full/empty barriers per slice let the next token's MMAs
+// start on a slice as soon as its codes are formed.
 //
 // Every mbarrier wait is bounded (kq_wait.cuh); a wait that gives up records
 // site 512 in the device status word and every role leaves its loop.
@@ -47,9 +49,11 @@ using namespace tc;
 enum : unsigned { kSiteTwoStage = 512u };
 
 constexpr int kMaxFactor = 256;
-constexpr int RT = 128;                 // rows of a tile (stage 1: rows (t, a); stage 2: lanes j)
+constexpr int RT = 128;                 // TMEM lanes: one slice of j
 constexpr int KCH = 64;                 // K elements per chunk: one 128-byte swizzle row of bf16
 constexpr int TILE = RT * KCH * 2;      // 16 KB: one bf16 tile [128][64]
+
+__host__ __device__ constexpr int slices(int n2) { return (n2 + RT - 1) / RT; }
 
 // 32 lanes x 32 bits, 8 columns: thread t <- lane t, registers = columns.
 __device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
@@ -81,38 +85,42 @@ __device__ __forceinline__ int round_code_ts(uint32_t ybits, float inv, int one)
 __device__ __forceinline__ uint32_t align1024(uint32_t a) { return (a + 1023u) & ~1023u; }
 
 // ============================================================================
-// Stage 1: Z^T hi/lo = split(P2^T X~'^T), one 128-wide slice of j per CTA
+// Stage 1: Z^T hi/lo = split(P2^T X~'^T)
 // ============================================================================
+constexpr int R1 = 64;                                     // rows (t, a) per tile: MMA N
+constexpr int XT = R1 * KCH * 2;                           // 8 KB: one x tile [64][64]
 constexpr int S1_THREADS = 512;
 constexpr int S1_NX = 4;                                   // loaded x stages
 constexpr int S1_NS = 2;                                   // hi/lo stages
-constexpr int S1_OFF_S = S1_NX * TILE;                     // 64 KB
-constexpr int S1_OFF_BAR = S1_OFF_S + S1_NS * 2 * TILE;    // 128 KB
+constexpr int SBOX = RT * 16 * 2;                          // 4 KB: one store box [128 j][16 a]
+constexpr int SG = 4 * SBOX;                               // 16 KB: hi and lo boxes of 32 rows
+constexpr int S1_OFF_S = S1_NX * XT;                       // 32 KB
+constexpr int S1_OFF_STG = S1_OFF_S + S1_NS * 2 * XT;      // 64 KB: two staging buffers
+constexpr int S1_OFF_BAR = S1_OFF_STG + 2 * SG;            // 96 KB
 constexpr int B1_XFULL = 0, B1_XEMPTY = S1_NX, B1_SFULL = 2 * S1_NX, B1_SEMPTY = 2 * S1_NX + S1_NS,
               B1_DFULL = 2 * S1_NX + 2 * S1_NS, B1_DEMPTY = B1_DFULL + 2, B1_DONE = B1_DEMPTY + 2,
               B1_COUNT = B1_DONE + 1;
 constexpr int S1_OFF_MISC = S1_OFF_BAR + 8 * B1_COUNT;     // TMEM base, abort flag
 constexpr int S1_SMEM = S1_OFF_MISC + 16 + 1024;           // + slack for 1024-byte alignment
 constexpr uint32_t S1_TMEM_COLS = 512;
-constexpr uint32_t S1_DCOL = 128;                          // D1 buffers at columns 128 and 256
+constexpr uint32_t S1_DCOL = 256;                          // A1 slices at 0 and 128; D1 [2 buffers][2 slices][64]
 static_assert(S1_SMEM <= 227 * 1024, "shared memory budget");
 
 template <bool SCALED>
 __global__ void __launch_bounds__(S1_THREADS, 1)
-    kq_two_stage_s1_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t *__restrict__ P2,
-                           const float *__restrict__ cinv, uint16_t *__restrict__ zhi,
-                           uint16_t *__restrict__ zlo, int64_t T, int n1, int n2, int ctas_per_slice,
-                           unsigned int *err) {
+    kq_two_stage_s1_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_shi,
+                           const __grid_constant__ CUtensorMap tmap_slo, const uint16_t *__restrict__ P2,
+                           const float *__restrict__ cinv, int64_t T, int n1, int n2, unsigned int *err) {
     extern __shared__ __align__(1024) unsigned char s1_raw[];
     const uint32_t raw_addr = smem_u32(s1_raw);
     const uint32_t sbase = align1024(raw_addr);
     unsigned char *smem = s1_raw + (sbase - raw_addr);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int jt = int(blockIdx.x) % ((n2 + RT - 1) / RT);     // slice of j
-    const int first = int(blockIdx.x) / ((n2 + RT - 1) / RT);  // first row tile
-    const int64_t rows = T * n1;
-    const int ntiles = int((rows + RT - 1) / RT);
-    const int KC = (n2 + KCH - 1) / KCH;                         // K chunks per row tile
+    const int J = slices(n2), Jp = RT * J;
+    const int rows = int(T * n1);                 // < 2^31 (checked by the entry)
+    const int ntiles = (rows + R1 - 1) / R1;
+    const int KC = (n2 + KCH - 1) / KCH;          // K chunks per tile
+    const int first = int(blockIdx.x), stride = int(gridDim.x);
     auto bar = [&](int i) -> uint32_t { return sbase + uint32_t(S1_OFF_BAR + 8 * i); };
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + S1_OFF_MISC + 4);
 
@@ -133,7 +141,11 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
         *s_abort = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_x);
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmap_x);
+        prefetch_tensormap(&tmap_shi);
+        prefetch_tensormap(&tmap_slo);
+    }
     if (warp == 1) {
         tmem_alloc(sbase + S1_OFF_MISC, S1_TMEM_COLS);
         tmem_relinquish();
@@ -144,20 +156,23 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + S1_OFF_MISC);
 
     if (warp >= 12) {
-        // A1 = this CTA's slice of P2^T into TMEM columns [0, KC * 32): lane m holds
-        // row j = 128 jt + m, K pairs (b, b + 1) packed per column; zero outside n2.
-        const int jg = RT * jt + 32 * (warp & 3) + lane;
-        const uint32_t taddr = tmem + (uint32_t(32 * (warp & 3)) << 16);
-        for (int c16 = 0; c16 < 2 * KC; ++c16) {
-            uint32_t w[16];
+        // A1 = P2^T into TMEM: slice s at columns [128 s, 128 s + 32 KC); lane m
+        // holds row j = 128 s + m, K pairs (b, b + 1) packed per column; zero
+        // outside n2 (rows j >= n2 give zero accumulators).
+        const uint32_t lanes = tmem + (uint32_t(32 * (warp & 3)) << 16);
+        for (int s = 0; s < J; ++s) {
+            const int jg = RT * s + 32 * (warp & 3) + lane;
+            for (int c16 = 0; c16 < 2 * KC; ++c16) {
+                uint32_t w[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int b = 32 * c16 + 2 * e;
-                const uint32_t v0 = (jg < n2 && b < n2) ? P2[b * n2 + jg] : 0u;
-                const uint32_t v1 = (jg < n2 && b + 1 < n2) ? P2[(b + 1) * n2 + jg] : 0u;
-                w[e] = v0 | (v1 << 16);
+                for (int e = 0; e < 16; ++e) {
+                    const int b = 32 * c16 + 2 * e;
+                    const uint32_t v0 = (jg < n2 && b < n2) ? P2[b * n2 + jg] : 0u;
+                    const uint32_t v1 = (jg < n2 && b + 1 < n2) ? P2[(b + 1) * n2 + jg] : 0u;
+                    w[e] = v0 | (v1 << 16);
+                }
+                tmem_st_32x32b_x16(lanes + uint32_t(RT * s + 16 * c16), w);
             }
-            tmem_st_32x32b_x16(taddr + 16 * c16, w);
         }
         tmem_wait_st();
     }
@@ -166,24 +181,22 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
     tc_fence_after();
 
     if (warp == 0) {
-        // ---------------- TMA producer: x tiles [128 rows (t, a)] x [64 b] ----------------
+        // ---------------- TMA producer: x tiles [64 rows (t, a)] x [64 b] ----------------
         Ring r;
         int issued = 0;
-        for (int tile = first; tile < ntiles; tile += ctas_per_slice) {
-            bool ok = true;
+        bool ok = true;
+        for (int tile = first; tile < ntiles && ok; tile += stride)
             for (int kc = 0; kc < KC; ++kc, r.next(S1_NX)) {
                 ok = __all_sync(0xffffffffu, wait_bounded_err(bar(B1_XEMPTY + r.idx), r.phase ^ 1u, s_abort,
                                                               kSiteTwoStage, kWaitLimitNs, false, err));
                 if (!ok) break;
                 if (elect_one()) {
-                    mbar_arrive_expect_tx(bar(B1_XFULL + r.idx), TILE);
-                    tma_load_2d(sbase + uint32_t(r.idx * TILE), &tmap_x, kc * KCH, tile * RT, bar(B1_XFULL + r.idx));
+                    mbar_arrive_expect_tx(bar(B1_XFULL + r.idx), XT);
+                    tma_load_2d(sbase + uint32_t(r.idx * XT), &tmap_x, kc * KCH, tile * R1, bar(B1_XFULL + r.idx));
                 }
                 __syncwarp();
                 ++issued;
             }
-            if (!ok) break;
-        }
         // every load issued has landed before the CTA can exit
         Ring rd;
         for (int i = 0; i < issued; ++i, rd.next(S1_NX))
@@ -191,32 +204,34 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
                 wait_bounded_err(bar(B1_XFULL + rd.idx), rd.phase, s_abort, kSiteTwoStage, kWaitLimitNs, true, err);
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer: D1[j][row] = sum_b P2^T[j][b] x'[row][b] ----------------
-        constexpr uint32_t idesc = idesc_bf16_f32(128, RT);
+        // ---------------- MMA issuer: D1[s][j][row] = sum_b P2^T[128 s + j][b] x'[row][b] ----------------
+        constexpr uint32_t idesc = idesc_bf16_f32(128, R1);
         Ring rs, rd;
-        for (int tile = first; tile < ntiles; tile += ctas_per_slice, rd.next(2)) {
-            bool ok = wait_bounded_err(bar(B1_DEMPTY + rd.idx), rd.phase ^ 1u, s_abort, kSiteTwoStage,
-                                       kWaitLimitNs, false, err);
-            if (!__all_sync(0xffffffffu, ok)) break;
+        bool ok = true;
+        for (int tile = first; tile < ntiles && ok; tile += stride, rd.next(2)) {
+            ok = __all_sync(0xffffffffu, wait_bounded_err(bar(B1_DEMPTY + rd.idx), rd.phase ^ 1u, s_abort,
+                                                          kSiteTwoStage, kWaitLimitNs, false, err));
+            if (!ok) break;
             tc_fence_after();
-            const uint32_t d = tmem + S1_DCOL + 128u * rd.idx;
             for (int kc = 0; kc < KC; ++kc, rs.next(SCALED ? S1_NS : S1_NX)) {
                 ok = __all_sync(0xffffffffu, wait_bounded_err(bar((SCALED ? B1_SFULL : B1_XFULL) + rs.idx), rs.phase,
                                                               s_abort, kSiteTwoStage, kWaitLimitNs, false, err));
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t hi = SCALED ? sbase + uint32_t(S1_OFF_S + rs.idx * 2 * TILE)
-                                           : sbase + uint32_t(rs.idx * TILE);
-                const uint32_t bh = sdesc_sw128_lo(hi), bl = sdesc_sw128_lo(hi + TILE);
+                const uint32_t hi = SCALED ? sbase + uint32_t(S1_OFF_S + rs.idx * 2 * XT) : sbase + uint32_t(rs.idx * XT);
+                const uint32_t bh = sdesc_sw128_lo(hi), bl = sdesc_sw128_lo(hi + XT);
                 if (elect_one()) {
+                    for (int s = 0; s < J; ++s) {
+                        const uint32_t d = tmem + S1_DCOL + 128u * rd.idx + uint32_t(R1 * s);
 #pragma unroll
-                    for (int kk = 0; kk < KCH / 16; ++kk) {
-                        const uint32_t a = tmem + uint32_t(32 * kc + 8 * kk);
-                        if ((kc | kk) != 0)
-                            mma_ts_split<1>(d, a, bh + 2 * kk, kSdescSw128Hi, idesc);
-                        else
-                            mma_ts_split<0>(d, a, bh + 2 * kk, kSdescSw128Hi, idesc);
-                        if (SCALED) mma_ts_split<1>(d, a, bl + 2 * kk, kSdescSw128Hi, idesc);
+                        for (int kk = 0; kk < KCH / 16; ++kk) {
+                            const uint32_t a = tmem + uint32_t(RT * s + 32 * kc + 8 * kk);
+                            if ((kc | kk) != 0)
+                                mma_ts_split<1>(d, a, bh + 2 * kk, kSdescSw128Hi, idesc);
+                            else
+                                mma_ts_split<0>(d, a, bh + 2 * kk, kSdescSw128Hi, idesc);
+                            if (SCALED) mma_ts_split<1>(d, a, bl + 2 * kk, kSdescSw128Hi, idesc);
+                        }
                     }
                     tc_commit(bar((SCALED ? B1_SEMPTY : B1_XEMPTY) + rs.idx));  // stage free once read
                 }
@@ -234,95 +249,142 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
     } else if (SCALED && warp >= 4 && warp < 12) {
         // ---------------- x' = x o cinv split into hi/lo bf16 tiles ----------------
         // Thread xt takes 16-byte chunk c = xt % 8 (8 values of b) of rows
-        // xt / 8 + 32 i; the swizzled offset is the same in every tile.
+        // xt / 8 and xt / 8 + 32; the swizzled offset is the same in every tile.
+        // cinv for the next chunk is loaded while this one is split.
         const int xt = tid - 128;
         const int c = xt & 7;
-        Ring rx, rs;
-        for (int tile = first; tile < ntiles; tile += ctas_per_slice) {
-            bool ok = true;
-            for (int kc = 0; kc < KC; ++kc, rx.next(S1_NX), rs.next(S1_NS)) {
-                ok = wait_bounded_err(bar(B1_XFULL + rx.idx), rx.phase, s_abort, kSiteTwoStage, kWaitLimitNs, false,
-                                      err);
-                ok = ok && wait_bounded_err(bar(B1_SEMPTY + rs.idx), rs.phase ^ 1u, s_abort, kSiteTwoStage,
-                                            kWaitLimitNs, false, err);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-                const unsigned char *src = smem + rx.idx * TILE;
-                unsigned char *dhi = smem + S1_OFF_S + rs.idx * 2 * TILE;
-                const int b = kc * KCH + 8 * c;
+        auto load_cinv = [&](int tile, int kc, float4 (&cv)[2][2]) {
+            const int b = kc * KCH + 8 * c;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = (xt >> 3) + 32 * i;
-                    const uint32_t off = uint32_t(r * 128 + ((c ^ (r & 7)) << 4));
-                    const uint4 v = *reinterpret_cast<const uint4 *>(src + off);
-                    float4 c0 = make_float4(0.f, 0.f, 0.f, 0.f), c1 = c0;
-                    if (b < n2) {  // chunks past n2 hold zeros from the load
-                        const int a = (tile * RT + r) % n1;
-                        const float4 *cp = reinterpret_cast<const float4 *>(cinv + a * n2 + b);
-                        c0 = __ldg(cp);
-                        c1 = __ldg(cp + 1);
-                    }
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                    const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                    uint32_t h[4], l[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        hi_lo_pair(__uint_as_float(w[e] << 16) * cs[2 * e],
-                                   __uint_as_float(w[e] & 0xFFFF0000u) * cs[2 * e + 1], h[e], l[e]);
-                    *reinterpret_cast<uint4 *>(dhi + off) = make_uint4(h[0], h[1], h[2], h[3]);
-                    *reinterpret_cast<uint4 *>(dhi + TILE + off) = make_uint4(l[0], l[1], l[2], l[3]);
-                }
-                fence_proxy_async_smem();  // tiles visible to the tensor cores
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(bar(B1_XEMPTY + rx.idx));
-                    mbar_arrive(bar(B1_SFULL + rs.idx));
+            for (int i = 0; i < 2; ++i) {
+                if (tile < ntiles && b < n2) {  // chunks past n2 hold zeros from the load
+                    const int a = (tile * R1 + (xt >> 3) + 32 * i) % n1;
+                    const float4 *cp = reinterpret_cast<const float4 *>(cinv + a * n2 + b);
+                    cv[i][0] = __ldg(cp);
+                    cv[i][1] = __ldg(cp + 1);
+                } else {
+                    cv[i][0] = cv[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
-            if (!ok) break;
+        };
+        Ring rx, rs;
+        float4 cur[2][2], nxt[2][2];
+        int tile = first, kc = 0;
+        load_cinv(tile, kc, cur);
+        while (tile < ntiles) {
+            int ntile = tile, nkc = kc + 1;
+            if (nkc == KC) {
+                nkc = 0;
+                ntile += stride;
+            }
+            load_cinv(ntile, nkc, nxt);
+            bool ok = wait_bounded_err(bar(B1_XFULL + rx.idx), rx.phase, s_abort, kSiteTwoStage, kWaitLimitNs, false,
+                                       err);
+            ok = ok && wait_bounded_err(bar(B1_SEMPTY + rs.idx), rs.phase ^ 1u, s_abort, kSiteTwoStage,
+                                        kWaitLimitNs, false, err);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const unsigned char *src = smem + rx.idx * XT;
+            unsigned char *dhi = smem + S1_OFF_S + rs.idx * 2 * XT;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int r = (xt >> 3) + 32 * i;
+                const uint32_t off = uint32_t(r * 128 + ((c ^ (r & 7)) << 4));
+                const uint4 v = *reinterpret_cast<const uint4 *>(src + off);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                const float cs[8] = {cur[i][0].x, cur[i][0].y, cur[i][0].z, cur[i][0].w,
+                                     cur[i][1].x, cur[i][1].y, cur[i][1].z, cur[i][1].w};
+                uint32_t h[4], l[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    hi_lo_pair(__uint_as_float(w[e] << 16) * cs[2 * e],
+                               __uint_as_float(w[e] & 0xFFFF0000u) * cs[2 * e + 1], h[e], l[e]);
+                *reinterpret_cast<uint4 *>(dhi + off) = make_uint4(h[0], h[1], h[2], h[3]);
+                *reinterpret_cast<uint4 *>(dhi + XT + off) = make_uint4(l[0], l[1], l[2], l[3]);
+            }
+            fence_proxy_async_smem();  // tiles visible to the tensor cores
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(B1_XEMPTY + rx.idx));
+                mbar_arrive(bar(B1_SFULL + rs.idx));
+            }
+            rx.next(S1_NX);
+            rs.next(S1_NS);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                cur[i][0] = nxt[i][0];
+                cur[i][1] = nxt[i][1];
+            }
+            tile = ntile;
+            kc = nkc;
         }
     } else if (warp >= 12) {
-        // ---------------- epilogue: D1 -> Z^T hi/lo in the workspace ----------------
-        // Thread = TMEM lane = j; each group of 8 consecutive rows of a tile is 8
-        // consecutive a of one token (n1 is a multiple of 16), stored as 16 bytes.
-        const int q = warp & 3;
-        const int jg = RT * jt + 32 * q + lane;
-        const bool jvalid = jg < n2;
+        // ---------------- epilogue: D1 -> Z^T hi/lo boxes -> TMA stores ----------------
+        // Thread = TMEM lane = j (within a slice).  Each 32-row half of a slice's
+        // accumulator becomes two [128 j][16 a] boxes of hi and two of lo (16
+        // consecutive rows stay in one token since n1 is a multiple of 16),
+        // staged in shared memory (two buffers) and stored by one thread.
+        const int q = warp & 3, et = tid - 384;
+        const int j = 32 * q + lane;
         Ring rd;
-        for (int tile = first; tile < ntiles; tile += ctas_per_slice, rd.next(2)) {
-            const bool ok = wait_bounded_err(bar(B1_DFULL + rd.idx), rd.phase, s_abort, kSiteTwoStage,
-                                             kWaitLimitNs, false, err);
-            if (!__all_sync(0xffffffffu, ok)) break;
+        int sb = 0;
+        for (int tile = first; tile < ntiles; tile += stride, rd.next(2)) {
+            const bool ok = wait_bounded_err(bar(B1_DFULL + rd.idx), rd.phase, s_abort, kSiteTwoStage, kWaitLimitNs,
+                                             false, err);
+            if (named_barrier_any(1, 128, !__all_sync(0xffffffffu, ok))) break;  // leave together
             tc_fence_after();
-            const uint32_t col0 = tmem + (uint32_t(32 * q) << 16) + S1_DCOL + 128u * rd.idx;
-#pragma unroll 1
-            for (int cc = 0; cc < RT / 32; ++cc) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(col0 + 32 * cc, v);
-                tmem_wait_ld();
-                if (jvalid) {
-#pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const int R0 = tile * RT + 32 * cc + 8 * g;
-                        if (R0 < rows) {
-                            const int t = R0 / n1;
-                            const int a0 = R0 - t * n1;
-                            uint32_t h[4], l[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                hi_lo_pair(__uint_as_float(v[8 * g + 2 * e]), __uint_as_float(v[8 * g + 2 * e + 1]),
-                                           h[e], l[e]);
-                            const int64_t off = (int64_t(t) * n2 + jg) * n1 + a0;
-                            *reinterpret_cast<uint4 *>(zhi + off) = make_uint4(h[0], h[1], h[2], h[3]);
-                            *reinterpret_cast<uint4 *>(zlo + off) = make_uint4(l[0], l[1], l[2], l[3]);
-                        }
+            for (int s = 0; s < J; ++s)
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem + (uint32_t(32 * q) << 16) + S1_DCOL + 128u * rd.idx +
+                                           uint32_t(R1 * s + 32 * hf),
+                                       v);
+                    tmem_wait_ld();
+                    if (s == J - 1 && hf == 1) {  // this warp's last read of the buffer
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(B1_DEMPTY + rd.idx));
                     }
+                    uint32_t h[16], l[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        hi_lo_pair(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]), h[e], l[e]);
+                    if (et == 0) bulk_wait_read<1>();  // the stores that used this buffer have read it
+                    named_barrier_sync(2, 128);
+                    unsigned char *stg = smem + S1_OFF_STG + sb * SG;
+                    const int sw = (j >> 2) & 1;  // chunk order that spreads the 16-byte stores over all banks
+#pragma unroll
+                    for (int bx = 0; bx < 2; ++bx) {
+                        const uint4 h0 = make_uint4(h[8 * bx], h[8 * bx + 1], h[8 * bx + 2], h[8 * bx + 3]);
+                        const uint4 h1 = make_uint4(h[8 * bx + 4], h[8 * bx + 5], h[8 * bx + 6], h[8 * bx + 7]);
+                        const uint4 l0 = make_uint4(l[8 * bx], l[8 * bx + 1], l[8 * bx + 2], l[8 * bx + 3]);
+                        const uint4 l1 = make_uint4(l[8 * bx + 4], l[8 * bx + 5], l[8 * bx + 6], l[8 * bx + 7]);
+                        const uint32_t off = uint32_t(bx * SBOX + j * 32);
+                        const uint32_t o_first = sw ? 16u : 0u, o_second = sw ? 0u : 16u;
+                        *reinterpret_cast<uint4 *>(stg + off + o_first) = sw ? h1 : h0;
+                        *reinterpret_cast<uint4 *>(stg + 2 * SBOX + off + o_first) = sw ? l1 : l0;
+                        *reinterpret_cast<uint4 *>(stg + off + o_second) = sw ? h0 : h1;
+                        *reinterpret_cast<uint4 *>(stg + 2 * SBOX + off + o_second) = sw ? l0 : l1;
+                    }
+                    fence_proxy_async_smem();  // staging visible to the tensor stores
+                    named_barrier_sync(2, 128);
+                    if (et == 0) {
+                        const uint32_t sa = sbase + uint32_t(S1_OFF_STG + sb * SG);
+#pragma unroll
+                        for (int bx = 0; bx < 2; ++bx) {
+                            const int R = tile * R1 + 32 * hf + 16 * bx;
+                            if (R < rows) {
+                                const int t = R / n1, a0 = R - t * n1;
+                                const int y = t * Jp + RT * s;
+                                tma_store_2d(&tmap_shi, a0, y, sa + uint32_t(bx * SBOX));
+                                tma_store_2d(&tmap_slo, a0, y, sa + uint32_t(2 * SBOX + bx * SBOX));
+                            }
+                        }
+                        bulk_commit();
+                    }
+                    sb ^= 1;
                 }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B1_DEMPTY + rd.idx));
         }
+        if (et == 0) bulk_wait<0>();
     }
 
     tc_fence_before();
@@ -342,16 +404,15 @@ constexpr int S2_MAX_NA = 4;
 constexpr int S2_SMEM_MAX = 227 * 1024;
 
 // Shared-memory carve-up of the stage-2 kernel for one shape (byte offsets
-// from the 1024-aligned base).
+// from the 1024-aligned base) and its barrier indices.
 struct S2Layout {
     int n1, n2, J, AC, NA, NB, dcols;
     int off_b2, off_a, off_stg, off_bar, off_red, off_misc, smem;
-    // barriers
-    __host__ __device__ int AFULL() const { return 0; }
-    __host__ __device__ int AEMPTY() const { return NA; }
-    __host__ __device__ int DFULL() const { return 2 * NA; }
-    __host__ __device__ int DEMPTY() const { return 2 * NA + NB; }
-    __host__ __device__ int DONE() const { return 2 * NA + 2 * NB; }
+    __host__ __device__ int AFULL(int s) const { return s; }
+    __host__ __device__ int AEMPTY(int s) const { return NA + s; }
+    __host__ __device__ int DFULL(int b, int s) const { return 2 * NA + b * J + s; }
+    __host__ __device__ int DEMPTY(int b, int s) const { return 2 * NA + NB * J + b * J + s; }
+    __host__ __device__ int DONE() const { return 2 * NA + 2 * NB * J; }
     __host__ __device__ int nbar() const { return DONE() + 1; }
 };
 
@@ -359,7 +420,7 @@ __host__ __device__ inline S2Layout s2_layout(int n1, int n2) {
     S2Layout L{};
     L.n1 = n1;
     L.n2 = n2;
-    L.J = (n2 + RT - 1) / RT;
+    L.J = slices(n2);
     L.AC = (n1 + KCH - 1) / KCH;
     L.dcols = L.J * n1;
     L.NB = 2 * L.dcols <= 512 ? 2 : 1;
@@ -367,8 +428,8 @@ __host__ __device__ inline S2Layout s2_layout(int n1, int n2) {
     const int b2 = L.AC * n1 * 128;                 // P1^T chunks [n1 rows][128 B]
     L.off_a = (b2 + 1023) & ~1023;
     const int stg = n1 * n2 / 2;                    // one token's codes
-    const int fixed = 1024 /* alignment slack */ + L.off_a + stg + 8 * (2 * S2_MAX_NA + 5) + 64 + 16;
-    int na = (S2_SMEM_MAX - fixed) / (2 * TILE);
+    const int fixed = 1024 /* alignment slack */ + L.off_a + stg + 8 * (2 * S2_MAX_NA + 9) + 64 + 16;
+    const int na = (S2_SMEM_MAX - fixed) / (2 * TILE);
     L.NA = na > S2_MAX_NA ? S2_MAX_NA : na;
     L.off_stg = L.off_a + L.NA * 2 * TILE;
     L.off_bar = (L.off_stg + stg + 7) & ~7;
@@ -388,19 +449,20 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
     unsigned char *smem = s2_raw + (sbase - raw_addr);
     const S2Layout L = s2_layout(n1, n2);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n = n1 * n2;
+    const int n = n1 * n2, Jp = RT * L.J;
     auto bar = [&](int i) -> uint32_t { return sbase + uint32_t(L.off_bar + 8 * i); };
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L.off_misc + 4);
 
     if (tid == 0) {
         for (int s = 0; s < L.NA; ++s) {
-            mbar_init(bar(L.AFULL() + s), 1);
-            mbar_init(bar(L.AEMPTY() + s), 1);
+            mbar_init(bar(L.AFULL(s)), 1);
+            mbar_init(bar(L.AEMPTY(s)), 1);
         }
-        for (int b = 0; b < L.NB; ++b) {
-            mbar_init(bar(L.DFULL() + b), 1);
-            mbar_init(bar(L.DEMPTY() + b), 8);  // one arrive per epilogue warp
-        }
+        for (int b = 0; b < L.NB; ++b)
+            for (int s = 0; s < L.J; ++s) {
+                mbar_init(bar(L.DFULL(b, s)), 1);
+                mbar_init(bar(L.DEMPTY(b, s)), 8);  // one arrive per epilogue warp
+            }
         mbar_init(bar(L.DONE()), 1);
         *s_abort = 0;
         *reinterpret_cast<int *>(smem + L.off_misc + 8) = 1;  // `one` of the code rounding
@@ -434,20 +496,17 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
         int issued = 0;
         bool ok = true;
         for (int64_t t = blockIdx.x; t < T && ok; t += gridDim.x)
-            for (int jt = 0; jt < L.J && ok; ++jt)
+            for (int s = 0; s < L.J && ok; ++s)
                 for (int ac = 0; ac < L.AC; ++ac, r.next(L.NA)) {
-                    ok = wait_bounded_err(bar(L.AEMPTY() + r.idx), r.phase ^ 1u, s_abort, kSiteTwoStage,
-                                          kWaitLimitNs, false, err);
-                    if (!__all_sync(0xffffffffu, ok)) {
-                        ok = false;
-                        break;
-                    }
+                    ok = __all_sync(0xffffffffu, wait_bounded_err(bar(L.AEMPTY(r.idx)), r.phase ^ 1u, s_abort,
+                                                                  kSiteTwoStage, kWaitLimitNs, false, err));
+                    if (!ok) break;
                     if (elect_one()) {
                         const uint32_t dst = sbase + uint32_t(L.off_a + r.idx * 2 * TILE);
-                        const int y = int(t * n2) + RT * jt;
-                        mbar_arrive_expect_tx(bar(L.AFULL() + r.idx), 2 * TILE);
-                        tma_load_2d(dst, &tmap_zhi, ac * KCH, y, bar(L.AFULL() + r.idx));
-                        tma_load_2d(dst + TILE, &tmap_zlo, ac * KCH, y, bar(L.AFULL() + r.idx));
+                        const int y = int(t) * Jp + RT * s;
+                        mbar_arrive_expect_tx(bar(L.AFULL(r.idx)), 2 * TILE);
+                        tma_load_2d(dst, &tmap_zhi, ac * KCH, y, bar(L.AFULL(r.idx)));
+                        tma_load_2d(dst + TILE, &tmap_zlo, ac * KCH, y, bar(L.AFULL(r.idx)));
                     }
                     __syncwarp();
                     ++issued;
@@ -455,31 +514,25 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
         Ring rd;
         for (int i = 0; i < issued; ++i, rd.next(L.NA))
             if (i + L.NA >= issued)
-                wait_bounded_err(bar(L.AFULL() + rd.idx), rd.phase, s_abort, kSiteTwoStage, kWaitLimitNs, true, err);
+                wait_bounded_err(bar(L.AFULL(rd.idx)), rd.phase, s_abort, kSiteTwoStage, kWaitLimitNs, true, err);
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer: D2[j][i] = sum_a Z^T[j][a] P1^T[i][a] ----------------
+        // ---------------- MMA issuer: D2[s][j][i] = sum_a Z^T[128 s + j][a] P1^T[i][a] ----------------
         const uint32_t idesc = idesc_bf16_f32(128, n1);
         const uint32_t b2 = sdesc_sw128_lo(sbase + uint32_t(L.off_b2));
         Ring ra, rd;
         bool ok = true;
         for (int64_t t = blockIdx.x; t < T && ok; t += gridDim.x, rd.next(L.NB)) {
-            ok = wait_bounded_err(bar(L.DEMPTY() + rd.idx), rd.phase ^ 1u, s_abort, kSiteTwoStage, kWaitLimitNs,
-                                  false, err);
-            if (!__all_sync(0xffffffffu, ok)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            for (int jt = 0; jt < L.J && ok; ++jt) {
-                const uint32_t d = tmem + uint32_t(rd.idx * L.dcols + jt * n1);
+            for (int s = 0; s < L.J && ok; ++s) {
+                ok = __all_sync(0xffffffffu, wait_bounded_err(bar(L.DEMPTY(rd.idx, s)), rd.phase ^ 1u, s_abort,
+                                                              kSiteTwoStage, kWaitLimitNs, false, err));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t d = tmem + uint32_t(rd.idx * L.dcols + s * n1);
                 for (int ac = 0; ac < L.AC; ++ac, ra.next(L.NA)) {
-                    ok = wait_bounded_err(bar(L.AFULL() + ra.idx), ra.phase, s_abort, kSiteTwoStage, kWaitLimitNs,
-                                          false, err);
-                    if (!__all_sync(0xffffffffu, ok)) {
-                        ok = false;
-                        break;
-                    }
+                    ok = __all_sync(0xffffffffu, wait_bounded_err(bar(L.AFULL(ra.idx)), ra.phase, s_abort,
+                                                                  kSiteTwoStage, kWaitLimitNs, false, err));
+                    if (!ok) break;
                     tc_fence_after();
                     const uint32_t ah = sdesc_sw128_lo(sbase + uint32_t(L.off_a + ra.idx * 2 * TILE));
                     const uint32_t al = ah + uint32_t(TILE >> 4);
@@ -495,14 +548,14 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
                                 mma_ss_split<0>(d, dh, bc + 2 * kk, kSdescSw128Hi, idesc);
                             mma_ss_split<1>(d, dl, bc + 2 * kk, kSdescSw128Hi, idesc);
                         }
-                        tc_commit(bar(L.AEMPTY() + ra.idx));
+                        tc_commit(bar(L.AEMPTY(ra.idx)));
                     }
                     __syncwarp();
                 }
+                if (!ok) break;
+                if (elect_one()) tc_commit(bar(L.DFULL(rd.idx, s)));  // this slice of the token is ready
+                __syncwarp();
             }
-            if (!ok) break;
-            if (elect_one()) tc_commit(bar(L.DFULL() + rd.idx));
-            __syncwarp();
         }
         if (elect_one()) tc_commit(bar(L.DONE()));
         __syncwarp();
@@ -510,8 +563,8 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
         __syncwarp();
     } else if (warp >= 4) {
         // ---------------- epilogue: absmax, codes, packing, one bulk store per token ----------------
-        // Thread = TMEM lane = column j of a 128-lane block; warpgroup ew takes
-        // columns (i) [ew h, ew h + h) of every block, h = n1 / 2.
+        // Thread = TMEM lane = column j of a slice; warpgroup ew takes columns
+        // (i) [ew h, ew h + h) of every slice, h = n1 / 2, in runs of up to 32.
         const int ew = (warp - 4) >> 2, q = warp & 3, et = tid - 128;
         const int h = n1 / 2;
         const int one = *reinterpret_cast<volatile int *>(smem + L.off_misc + 8);
@@ -520,62 +573,81 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
         Ring rd;
         int par = 0;
         for (int64_t t = blockIdx.x; t < T; t += gridDim.x, rd.next(L.NB), par ^= 1) {
-            bool ok = wait_bounded_err(bar(L.DFULL() + rd.idx), rd.phase, s_abort, kSiteTwoStage, kWaitLimitNs,
-                                       false, err);
-            ok = __all_sync(0xffffffffu, ok);
-            if (named_barrier_any(3, 256, !ok)) break;  // all epilogue warps leave together
-            tc_fence_after();
             const uint32_t lanes = tmem + (uint32_t(32 * q) << 16) + uint32_t(rd.idx * L.dcols + ew * h);
-            // pass 1: absmax over the valid lanes
+            // pass 1: absmax over the valid lanes, slice by slice as they complete
             float m = 0.0f;
-            for (int jt = 0; jt < L.J; ++jt) {
-                const bool valid = RT * jt + 32 * q + lane < n2;
-                for (int c8 = 0; c8 < h; c8 += 8) {
-                    uint32_t v[8];
-                    tmem_ld_32x32b_x8(lanes + uint32_t(jt * n1 + c8), v);
+            bool ok = true;
+            for (int s = 0; s < L.J; ++s) {
+                ok = ok && wait_bounded_err(bar(L.DFULL(rd.idx, s)), rd.phase, s_abort, kSiteTwoStage, kWaitLimitNs,
+                                            false, err);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const bool valid = RT * s + 32 * q + lane < n2;
+                for (int c = 0; c < h; c += 32) {
+                    const int cnt = h - c < 32 ? h - c : 32;  // a multiple of 8
+                    uint32_t v[4][8];
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        if (8 * g < cnt) tmem_ld_32x32b_x8(lanes + uint32_t(s * n1 + c + 8 * g), v[g]);
                     tmem_wait_ld();
                     if (valid) {
 #pragma unroll
-                        for (int e = 0; e < 8; e += 2)
-                            m = fmax3(m, fabsf(__uint_as_float(v[e])), fabsf(__uint_as_float(v[e + 1])));
+                        for (int g = 0; g < 4; ++g)
+                            if (8 * g < cnt) {
+#pragma unroll
+                                for (int e = 0; e < 8; e += 2)
+                                    m = fmax3(m, fabsf(__uint_as_float(v[g][e])), fabsf(__uint_as_float(v[g][e + 1])));
+                            }
                     }
                 }
             }
             const unsigned mw = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
             if (lane == 0) red[8 * par + (warp - 4)] = __uint_as_float(mw);
             if (et == 0) bulk_wait_read<0>();  // the previous token's codes have left the staging buffer
-            named_barrier_sync(1, 256);
+            if (named_barrier_any(1, 256, !ok)) break;  // all epilogue warps leave together
             float M = red[8 * par];
 #pragma unroll
             for (int w = 1; w < 8; ++w) M = fmaxf(M, red[8 * par + w]);
-            const float s = alpha * M * (1.0f / 7.0f);
-            const float inv = s > 0.0f ? fminf(__fdividef(1.0f, s), 3.0e38f) : 0.0f;
-            if (et == 0) scale_out[t] = s;
+            const float sc = alpha * M * (1.0f / 7.0f);
+            const float inv = sc > 0.0f ? fminf(__fdividef(1.0f, sc), 3.0e38f) : 0.0f;
+            if (et == 0) scale_out[t] = sc;
             // pass 2: codes; lanes j .. j + 7 gather one 32-bit word of row i
-            for (int jt = 0; jt < L.J; ++jt) {
-                const int jg = RT * jt + 32 * q + lane;
+            for (int s = 0; s < L.J; ++s) {
+                const int jg = RT * s + 32 * q + lane;
                 const bool store = jg < n2 && (lane & 7) == 0;
-                for (int c8 = 0; c8 < h; c8 += 8) {
-                    uint32_t v[8];
-                    tmem_ld_32x32b_x8(lanes + uint32_t(jt * n1 + c8), v);
-                    tmem_wait_ld();
+                for (int c = 0; c < h; c += 32) {
+                    const int cnt = h - c < 32 ? h - c : 32;
+                    uint32_t v[4][8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int code = round_code_ts(v[e], inv, one);
-                        const int nb = __shfl_xor_sync(0xffffffffu, code, 1);
-                        const uint32_t b8 = pack_s4x2(nb, code, 0u);  // even lane: own code low, neighbour high
-                        const uint32_t b16 = b8 | (__shfl_xor_sync(0xffffffffu, b8, 2) << 8);
-                        const uint32_t b32 = b16 | (__shfl_xor_sync(0xffffffffu, b16, 4) << 16);
-                        if (store) {
-                            const int i = ew * h + c8 + e;
-                            *reinterpret_cast<uint32_t *>(stg + ((i * n2 + jg) >> 1)) = b32;
-                        }
+                    for (int g = 0; g < 4; ++g)
+                        if (8 * g < cnt) tmem_ld_32x32b_x8(lanes + uint32_t(s * n1 + c + 8 * g), v[g]);
+                    tmem_wait_ld();
+                    if (c + 32 >= h) {  // this warp's last read of the slice
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(L.DEMPTY(rd.idx, s)));
                     }
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        if (8 * g < cnt) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const int code = round_code_ts(v[g][e], inv, one);
+                                const int nb = __shfl_xor_sync(0xffffffffu, code, 1);
+                                const uint32_t b8 = pack_s4x2(nb, code, 0u);  // even lane: own code low, neighbour high
+                                const uint32_t b16 = b8 | (__shfl_xor_sync(0xffffffffu, b8, 2) << 8);
+                                const uint32_t b32 = b16 | (__shfl_xor_sync(0xffffffffu, b16, 4) << 16);
+                                if (store) {
+                                    const int i = ew * h + c + 8 * g + e;
+                                    *reinterpret_cast<uint32_t *>(stg + ((i * n2 + jg) >> 1)) = b32;
+                                }
+                            }
+                        }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L.DEMPTY() + rd.idx));
             fence_proxy_async_smem();  // staging writes visible to the bulk copy
             named_barrier_sync(2, 256);
             if (et == 0) {
@@ -595,15 +667,16 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
     }
 }
 
-CUresult encode_bf16_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows) {
+CUresult encode_bf16_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                        uint32_t box_rows, CUtensorMapSwizzle swizzle) {
     PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
     if (!encode) return CUDA_ERROR_NOT_SUPPORTED;
     const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
     const cuuint64_t stride[1] = {cuuint64_t(cols * 2)};
-    const cuuint32_t box[2] = {cuuint32_t(KCH), cuuint32_t(RT)};
+    const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1u, 1u};
     return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, stride, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
@@ -613,7 +686,9 @@ bool two_stage_supports(int n1, int n2) {
     return n1 >= 16 && n2 >= 16 && n1 <= kMaxFactor && n2 <= kMaxFactor && n1 % 16 == 0 && n2 % 16 == 0;
 }
 
-uint64_t two_stage_workspace_bytes(int64_t T, int n1, int n2) { return uint64_t(T) * uint64_t(n1) * n2 * 4; }
+uint64_t two_stage_workspace_bytes(int64_t T, int n1, int n2) {
+    return uint64_t(T) * uint64_t(n1) * uint64_t(RT * slices(n2)) * 4;
+}
 
 cudaError_t launch_two_stage(const LaunchArgs &a, void *workspace) {
     static std::once_flag once[64];
@@ -639,33 +714,33 @@ cudaError_t launch_two_stage(const LaunchArgs &a, void *workspace) {
     cudaError_t e = device_error_word(a.device, &err);
     if (e != cudaSuccess) return e;
 
-    const int64_t n = int64_t(a.n1) * a.n2;
+    const uint64_t zrows = uint64_t(a.T) * uint64_t(RT * slices(a.n2));  // Z^T rows, padded per token
     uint16_t *zhi = static_cast<uint16_t *>(workspace);
-    uint16_t *zlo = zhi + a.T * n;
-    CUtensorMap tx, th, tl;
-    if (encode_bf16_2d(&tx, a.x, uint64_t(a.n2), uint64_t(a.T) * a.n1) != CUDA_SUCCESS ||
-        encode_bf16_2d(&th, zhi, uint64_t(a.n1), uint64_t(a.T) * a.n2) != CUDA_SUCCESS ||
-        encode_bf16_2d(&tl, zlo, uint64_t(a.n1), uint64_t(a.T) * a.n2) != CUDA_SUCCESS)
+    uint16_t *zlo = zhi + zrows * uint64_t(a.n1);
+    CUtensorMap tx, shi, slo, lhi, llo;
+    if (encode_bf16_2d(&tx, a.x, uint64_t(a.n2), uint64_t(a.T) * a.n1, KCH, R1, CU_TENSOR_MAP_SWIZZLE_128B) !=
+            CUDA_SUCCESS ||
+        encode_bf16_2d(&shi, zhi, uint64_t(a.n1), zrows, 16, RT, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
+        encode_bf16_2d(&slo, zlo, uint64_t(a.n1), zrows, 16, RT, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
+        encode_bf16_2d(&lhi, zhi, uint64_t(a.n1), zrows, KCH, RT, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+        encode_bf16_2d(&llo, zlo, uint64_t(a.n1), zrows, KCH, RT, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
 
-    // stage 1: J slices of j, each walked by ctas_per_slice CTAs over the row tiles
-    const int J = (a.n2 + RT - 1) / RT;
-    const int64_t ntiles = (a.T * a.n1 + RT - 1) / RT;
-    int per = a.num_sms / J;
-    if (per < 1) per = 1;
-    if (per > ntiles) per = int(ntiles);
+    // stage 1: persistent CTAs over 64-row tiles
+    const int64_t ntiles = (a.T * a.n1 + R1 - 1) / R1;
+    const int64_t g1 = ntiles < a.num_sms ? ntiles : a.num_sms;
     if (a.cinv)
-        kq_two_stage_s1_kernel<true><<<unsigned(J * per), S1_THREADS, S1_SMEM, a.stream>>>(
-            tx, a.P2, a.cinv, zhi, zlo, a.T, a.n1, a.n2, per, err);
+        kq_two_stage_s1_kernel<true><<<unsigned(g1), S1_THREADS, S1_SMEM, a.stream>>>(tx, shi, slo, a.P2, a.cinv, a.T,
+                                                                                      a.n1, a.n2, err);
     else
-        kq_two_stage_s1_kernel<false><<<unsigned(J * per), S1_THREADS, S1_SMEM, a.stream>>>(
-            tx, a.P2, nullptr, zhi, zlo, a.T, a.n1, a.n2, per, err);
+        kq_two_stage_s1_kernel<false><<<unsigned(g1), S1_THREADS, S1_SMEM, a.stream>>>(tx, shi, slo, a.P2, nullptr,
+                                                                                       a.T, a.n1, a.n2, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
     // stage 2: one CTA per SM, tokens strided
     const int64_t g2 = a.T < a.num_sms ? a.T : a.num_sms;
-    kq_two_stage_s2_kernel<<<unsigned(g2), S2_THREADS, L.smem, a.stream>>>(th, tl, a.P1, a.alpha, a.q_out,
+    kq_two_stage_s2_kernel<<<unsigned(g2), S2_THREADS, L.smem, a.stream>>>(lhi, llo, a.P1, a.alpha, a.q_out,
                                                                            a.scale_out, a.T, a.n1, a.n2, err);
     return cudaGetLastError();
 }

@@ -156,6 +156,7 @@ def test_two_stage_validation(kq):
     T, n1, n2 = 4, 256, 256
     need = kq.kq_two_stage_workspace_bytes(T, n1, n2)
     assert need == 4 * T * n1 * n2
+    assert kq.kq_two_stage_workspace_bytes(3, 64, 144) == 4 * 3 * 64 * 256   # Z^T rows padded to 128-row slices
     assert kq.kq_two_stage_workspace_bytes(0, 256, 256) == 0 and kq.kq_two_stage_workspace_bytes(-3, 16, 16) == 0
     ok = (x, P1, P2, c, 0.9, q, s_, w, need)
     assert f(*ok[:8], need, -1, n1, n2, None) == kq.KQ_ERR_SHAPE
