@@ -17,19 +17,26 @@
 // is known, so the codes leave from the stage-2 kernel and neither Y~ nor an
 // fp32 intermediate is ever written.  Factors are multiples of 16 up to 256.
 //
-// Stage 1 (512 threads, persistent over tiles of 64 rows (t, a)): warp 0 TMA
+// Stage 1 (640 threads, persistent over tiles of 64 rows (t, a)): warp 0 TMA
 // loads of x tiles [64 rows] x [64 b]; warp 1 TMEM allocation and MMA issue
 // (A = P2^T in 128-row slices of j, resident in TMEM; B = the x' hi and lo
 // tiles; N = 64); warps 4-11 split x o cinv into hi/lo tiles, with cinv loaded
 // one chunk ahead (without cinv the MMA reads the loaded tile as is); warps
-// 12-15 write P2^T into TMEM, then split each accumulator into Z^T hi/lo and
-// store it with TMA tensor stores of [128 j] x [16 a] boxes.
+// 12-19 (two warpgroups) write P2^T into TMEM, then split each accumulator
+// into Z^T hi/lo and store it with TMA tensor stores of [128 j] x [16 a]
+// boxes, the warpgroups taking alternate 32-row halves.
+//
+// Lane order: TMEM lane m of slice s holds j = 128 s + lane_column(m) (within
+// each block of 32 lanes, lane 16 f + 8 s' + g holds column 4 g + 2 f + s'),
+// and Z^T row m of the slice is stored in that order, so that a stage-2
+// epilogue thread reading 16x256b rows holds four consecutive j of an output
+// row: two whole bytes of codes.
 //
 // Stage 2 (384 threads, persistent over tokens): warp 0 TMA loads of Z^T hi/lo
 // tiles [128 j] x [64 a]; warp 1 TMEM allocation and MMA issue (A = the Z^T
 // tiles, B = P1^T resident in shared memory, N = n1), one 128-lane slice of j
 // at a time; warps 4-11 the epilogue (two warpgroups, each half of every
-// slice's columns).  Full/empty barriers per slice let the next token's MMAs
+// slice's columns; two bytes of codes per thread and output row, no shuffles).  Full/empty barriers per slice let the next token's MMAs
 // start on a slice as soon as its codes are formed.
 //
 // Every mbarrier wait is bounded (kq_wait.cuh); a wait that gives up records
@@ -39,6 +46,7 @@
 #include "kq_common.cuh"
 #include "kq_internal.h"
 #include "kq_tc05_ptx.cuh"
+#include "kq_tile.cuh"
 #include "kq_wait.cuh"
 
 namespace kq {
@@ -55,11 +63,11 @@ constexpr int TILE = RT * KCH * 2;      // 16 KB: one bf16 tile [128][64]
 
 __host__ __device__ constexpr int slices(int n2) { return (n2 + RT - 1) / RT; }
 
-// 32 lanes x 32 bits, 8 columns: thread t <- lane t, registers = columns.
-__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                   "=r"(r[7])
+// 16 lanes x 256 bits, 8 columns: thread t gets lane t/4 in regs 0, 1 and lane
+// t/4 + 8 in regs 2, 3, columns 2 (t % 4) and 2 (t % 4) + 1.
+__device__ __forceinline__ void tmem_ld_16x256b_x1(uint32_t taddr, uint32_t (&r)[4]) {
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(taddr));
 }
 
@@ -89,14 +97,14 @@ __device__ __forceinline__ uint32_t align1024(uint32_t a) { return (a + 1023u) &
 // ============================================================================
 constexpr int R1 = 64;                                     // rows (t, a) per tile: MMA N
 constexpr int XT = R1 * KCH * 2;                           // 8 KB: one x tile [64][64]
-constexpr int S1_THREADS = 512;
+constexpr int S1_THREADS = 640;
 constexpr int S1_NX = 4;                                   // loaded x stages
 constexpr int S1_NS = 2;                                   // hi/lo stages
 constexpr int SBOX = RT * 16 * 2;                          // 4 KB: one store box [128 j][16 a]
 constexpr int SG = 4 * SBOX;                               // 16 KB: hi and lo boxes of 32 rows
 constexpr int S1_OFF_S = S1_NX * XT;                       // 32 KB
-constexpr int S1_OFF_STG = S1_OFF_S + S1_NS * 2 * XT;      // 64 KB: two staging buffers
-constexpr int S1_OFF_BAR = S1_OFF_STG + 2 * SG;            // 96 KB
+constexpr int S1_OFF_STG = S1_OFF_S + S1_NS * 2 * XT;      // 64 KB: two staging buffers per epilogue warpgroup
+constexpr int S1_OFF_BAR = S1_OFF_STG + 4 * SG;            // 128 KB
 constexpr int B1_XFULL = 0, B1_XEMPTY = S1_NX, B1_SFULL = 2 * S1_NX, B1_SEMPTY = 2 * S1_NX + S1_NS,
               B1_DFULL = 2 * S1_NX + 2 * S1_NS, B1_DEMPTY = B1_DFULL + 2, B1_DONE = B1_DEMPTY + 2,
               B1_COUNT = B1_DONE + 1;
@@ -135,7 +143,7 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(B1_DFULL + b), 1);
-            mbar_init(bar(B1_DEMPTY + b), 4);
+            mbar_init(bar(B1_DEMPTY + b), 8);  // one arrive per epilogue warp
         }
         mbar_init(bar(B1_DONE), 1);
         *s_abort = 0;
@@ -157,11 +165,12 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
 
     if (warp >= 12) {
         // A1 = P2^T into TMEM: slice s at columns [128 s, 128 s + 32 KC); lane m
-        // holds row j = 128 s + m, K pairs (b, b + 1) packed per column; zero
-        // outside n2 (rows j >= n2 give zero accumulators).
+        // holds row j = 128 s + lane_column(m), K pairs (b, b + 1) packed per
+        // column; zero outside n2 (rows j >= n2 give zero accumulators).
+        // Warpgroup 12-15 writes slice 0, 16-19 slice 1.
         const uint32_t lanes = tmem + (uint32_t(32 * (warp & 3)) << 16);
-        for (int s = 0; s < J; ++s) {
-            const int jg = RT * s + 32 * (warp & 3) + lane;
+        for (int s = (warp - 12) >> 2; s < J; s += 2) {
+            const int jg = RT * s + tile::lane_column(32 * (warp & 3) + lane);
             for (int c16 = 0; c16 < 2 * KC; ++c16) {
                 uint32_t w[16];
 #pragma unroll
@@ -323,23 +332,24 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
         // accumulator becomes two [128 j][16 a] boxes of hi and two of lo (16
         // consecutive rows stay in one token since n1 is a multiple of 16),
         // staged in shared memory (two buffers) and stored by one thread.
-        const int q = warp & 3, et = tid - 384;
+        const int ew = (warp - 12) >> 2, q = warp & 3, et = tid - 384 - 128 * ew;
         const int j = 32 * q + lane;
+        const uint32_t nb_leave = 1u + uint32_t(ew), nb_stage = 3u + uint32_t(ew);
         Ring rd;
         int sb = 0;
         for (int tile = first; tile < ntiles; tile += stride, rd.next(2)) {
             const bool ok = wait_bounded_err(bar(B1_DFULL + rd.idx), rd.phase, s_abort, kSiteTwoStage, kWaitLimitNs,
                                              false, err);
-            if (named_barrier_any(1, 128, !__all_sync(0xffffffffu, ok))) break;  // leave together
+            if (named_barrier_any(nb_leave, 128, !__all_sync(0xffffffffu, ok))) break;  // leave together
             tc_fence_after();
             for (int s = 0; s < J; ++s)
-                for (int hf = 0; hf < 2; ++hf) {
+                for (int hf = ew; hf < 2; hf += 2) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tmem + (uint32_t(32 * q) << 16) + S1_DCOL + 128u * rd.idx +
                                            uint32_t(R1 * s + 32 * hf),
                                        v);
                     tmem_wait_ld();
-                    if (s == J - 1 && hf == 1) {  // this warp's last read of the buffer
+                    if (s == J - 1) {  // this warp's last read of the buffer
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar(B1_DEMPTY + rd.idx));
@@ -349,8 +359,8 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
                     for (int e = 0; e < 16; ++e)
                         hi_lo_pair(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]), h[e], l[e]);
                     if (et == 0) bulk_wait_read<1>();  // the stores that used this buffer have read it
-                    named_barrier_sync(2, 128);
-                    unsigned char *stg = smem + S1_OFF_STG + sb * SG;
+                    named_barrier_sync(nb_stage, 128);
+                    unsigned char *stg = smem + S1_OFF_STG + (2 * ew + sb) * SG;
                     const int sw = (j >> 2) & 1;  // chunk order that spreads the 16-byte stores over all banks
 #pragma unroll
                     for (int bx = 0; bx < 2; ++bx) {
@@ -366,9 +376,9 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
                         *reinterpret_cast<uint4 *>(stg + 2 * SBOX + off + o_second) = sw ? l0 : l1;
                     }
                     fence_proxy_async_smem();  // staging visible to the tensor stores
-                    named_barrier_sync(2, 128);
+                    named_barrier_sync(nb_stage, 128);
                     if (et == 0) {
-                        const uint32_t sa = sbase + uint32_t(S1_OFF_STG + sb * SG);
+                        const uint32_t sa = sbase + uint32_t(S1_OFF_STG + (2 * ew + sb) * SG);
 #pragma unroll
                         for (int bx = 0; bx < 2; ++bx) {
                             const int R = tile * R1 + 32 * hf + 16 * bx;
@@ -563,9 +573,14 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
         __syncwarp();
     } else if (warp >= 4) {
         // ---------------- epilogue: absmax, codes, packing, one bulk store per token ----------------
-        // Thread = TMEM lane = column j of a slice; warpgroup ew takes columns
-        // (i) [ew h, ew h + h) of every slice, h = n1 / 2, in runs of up to 32.
+        // Warpgroup ew takes columns (i) [ew h, ew h + h) of every slice, h = n1 / 2,
+        // in runs of up to 32.  With 16x256b loads of both 16-lane halves of its
+        // warp's lanes, thread (g, cp) = (lane / 4, lane % 4) holds lanes
+        // 32 q + g + {0, 8, 16, 24}, i.e. (by the lane order stage 1 wrote) the
+        // four consecutive columns j = 128 s + 32 q + 4 g + {0, 1, 2, 3}, for the
+        // rows i = 8 u + 2 cp + {0, 1} of each run of 8: two bytes of codes each.
         const int ew = (warp - 4) >> 2, q = warp & 3, et = tid - 128;
+        const int g = lane >> 2, cp = lane & 3;
         const int h = n1 / 2;
         const int one = *reinterpret_cast<volatile int *>(smem + L.off_misc + 8);
         float *red = reinterpret_cast<float *>(smem + L.off_red);
@@ -574,7 +589,7 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
         int par = 0;
         for (int64_t t = blockIdx.x; t < T; t += gridDim.x, rd.next(L.NB), par ^= 1) {
             const uint32_t lanes = tmem + (uint32_t(32 * q) << 16) + uint32_t(rd.idx * L.dcols + ew * h);
-            // pass 1: absmax over the valid lanes, slice by slice as they complete
+            // pass 1: absmax over the valid columns, slice by slice as they complete
             float m = 0.0f;
             bool ok = true;
             for (int s = 0; s < L.J; ++s) {
@@ -585,21 +600,24 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const bool valid = RT * s + 32 * q + lane < n2;
+                const bool valid = RT * s + 32 * q + 4 * g < n2;
                 for (int c = 0; c < h; c += 32) {
                     const int cnt = h - c < 32 ? h - c : 32;  // a multiple of 8
-                    uint32_t v[4][8];
+                    uint32_t ra[4][4], rb[4][4];
 #pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        if (8 * g < cnt) tmem_ld_32x32b_x8(lanes + uint32_t(s * n1 + c + 8 * g), v[g]);
+                    for (int u = 0; u < 4; ++u)
+                        if (8 * u < cnt) {
+                            tmem_ld_16x256b_x1(lanes + uint32_t(s * n1 + c + 8 * u), ra[u]);
+                            tmem_ld_16x256b_x1(lanes + (16u << 16) + uint32_t(s * n1 + c + 8 * u), rb[u]);
+                        }
                     tmem_wait_ld();
                     if (valid) {
 #pragma unroll
-                        for (int g = 0; g < 4; ++g)
-                            if (8 * g < cnt) {
+                        for (int u = 0; u < 4; ++u)
+                            if (8 * u < cnt) {
 #pragma unroll
-                                for (int e = 0; e < 8; e += 2)
-                                    m = fmax3(m, fabsf(__uint_as_float(v[g][e])), fabsf(__uint_as_float(v[g][e + 1])));
+                                for (int e = 0; e < 4; ++e)
+                                    m = fmax3(m, fabsf(__uint_as_float(ra[u][e])), fabsf(__uint_as_float(rb[u][e])));
                             }
                     }
                 }
@@ -614,16 +632,19 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
             const float sc = alpha * M * (1.0f / 7.0f);
             const float inv = sc > 0.0f ? fminf(__fdividef(1.0f, sc), 3.0e38f) : 0.0f;
             if (et == 0) scale_out[t] = sc;
-            // pass 2: codes; lanes j .. j + 7 gather one 32-bit word of row i
+            // pass 2: codes, two bytes (columns 4 g .. 4 g + 3) per row i
             for (int s = 0; s < L.J; ++s) {
-                const int jg = RT * s + 32 * q + lane;
-                const bool store = jg < n2 && (lane & 7) == 0;
+                const int jb = RT * s + 32 * q + 4 * g;
+                const bool store = jb < n2;
                 for (int c = 0; c < h; c += 32) {
                     const int cnt = h - c < 32 ? h - c : 32;
-                    uint32_t v[4][8];
+                    uint32_t ra[4][4], rb[4][4];
 #pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        if (8 * g < cnt) tmem_ld_32x32b_x8(lanes + uint32_t(s * n1 + c + 8 * g), v[g]);
+                    for (int u = 0; u < 4; ++u)
+                        if (8 * u < cnt) {
+                            tmem_ld_16x256b_x1(lanes + uint32_t(s * n1 + c + 8 * u), ra[u]);
+                            tmem_ld_16x256b_x1(lanes + (16u << 16) + uint32_t(s * n1 + c + 8 * u), rb[u]);
+                        }
                     tmem_wait_ld();
                     if (c + 32 >= h) {  // this warp's last read of the slice
                         tc_fence_before();
@@ -631,18 +652,17 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
                         if (lane == 0) mbar_arrive(bar(L.DEMPTY(rd.idx, s)));
                     }
 #pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        if (8 * g < cnt) {
+                    for (int u = 0; u < 4; ++u)
+                        if (8 * u < cnt) {
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const int code = round_code_ts(v[g][e], inv, one);
-                                const int nb = __shfl_xor_sync(0xffffffffu, code, 1);
-                                const uint32_t b8 = pack_s4x2(nb, code, 0u);  // even lane: own code low, neighbour high
-                                const uint32_t b16 = b8 | (__shfl_xor_sync(0xffffffffu, b8, 2) << 8);
-                                const uint32_t b32 = b16 | (__shfl_xor_sync(0xffffffffu, b16, 4) << 16);
+                            for (int d = 0; d < 2; ++d) {
+                                const uint32_t hi = pack_s4x2(round_code_ts(rb[u][2 + d], inv, one),
+                                                              round_code_ts(rb[u][d], inv, one), 0u);
+                                const uint32_t w = pack_s4x2(round_code_ts(ra[u][2 + d], inv, one),
+                                                             round_code_ts(ra[u][d], inv, one), hi);
                                 if (store) {
-                                    const int i = ew * h + c + 8 * g + e;
-                                    *reinterpret_cast<uint32_t *>(stg + ((i * n2 + jg) >> 1)) = b32;
+                                    const int i = ew * h + c + 8 * u + 2 * cp + d;
+                                    *reinterpret_cast<uint16_t *>(stg + ((i * n2 + jb) >> 1)) = uint16_t(w);
                                 }
                             }
                         }
