@@ -20,11 +20,12 @@
 // Stage 1 (640 threads, persistent over tiles of 64 rows (t, a)): warp 0 TMA
 // loads of x tiles [64 rows] x [64 b]; warp 1 TMEM allocation and MMA issue
 // (A = P2^T in 128-row slices of j, resident in TMEM; B = the x' hi and lo
-// tiles; N = 64); warps 4-11 split x o cinv into hi/lo tiles, with cinv loaded
-// one chunk ahead (without cinv the MMA reads the loaded tile as is); warps
+// tiles; N = 64); warps 4-11 split x o cinv into hi/lo tiles, cinv tiles
+// arriving by TMA with the x tiles (without cinv the MMA reads the loaded x
+// tile as is); warps
 // 12-19 (two warpgroups) write P2^T into TMEM, then split each accumulator
-// into Z^T hi/lo and store it with TMA tensor stores of [128 j] x [16 a]
-// boxes, the warpgroups taking alternate 32-row halves.
+// into Z^T hi/lo and store it with per-warp TMA tensor stores of [32 j] x
+// [16 a] boxes, the warpgroups taking alternate 32-row halves.
 //
 // Lane order: TMEM lane m of slice s holds j = 128 s + lane_column(m) (within
 // each block of 32 lanes, lane 16 f + 8 s' + g holds column 4 g + 2 f + s'),
@@ -36,7 +37,8 @@
 // tiles [128 j] x [64 a]; warp 1 TMEM allocation and MMA issue (A = the Z^T
 // tiles, B = P1^T resident in shared memory, N = n1), one 128-lane slice of j
 // at a time; warps 4-11 the epilogue (two warpgroups, each half of every
-// slice's columns; two bytes of codes per thread and output row, no shuffles).  Full/empty barriers per slice let the next token's MMAs
+// slice's columns; two bytes of codes per thread and output row, no shuffles,
+// stored straight to global memory).  Full/empty barriers per slice let the next token's MMAs
 // start on a slice as soon as its codes are formed.
 //
 // Every mbarrier wait is bounded (kq_wait.cuh); a wait that gives up records
@@ -71,6 +73,25 @@ __device__ __forceinline__ void tmem_ld_16x256b_x1(uint32_t taddr, uint32_t (&r)
                  : "r"(taddr));
 }
 
+// One run of up to 32 columns (cnt, a multiple of 8) of both 16-lane halves of a
+// warp's 32 lanes, in the 16x256b layout: ra[u] from lanes base + {g, g + 8},
+// rb[u] from lanes base + 16 + {g, g + 8}, columns 8 u + 2 (lane % 4) + {0, 1}.
+// Whole runs of 32 take one .x4 load per half; shorter ones .x1 loads.
+__device__ __forceinline__ void load_run(uint32_t taddr, int cnt, uint32_t (&ra)[4][4], uint32_t (&rb)[4][4]) {
+    if (cnt == 32) {
+        tmem_ld_16x256b_x4(taddr, *reinterpret_cast<uint32_t(*)[16]>(&ra[0][0]));
+        tmem_ld_16x256b_x4(taddr + (16u << 16), *reinterpret_cast<uint32_t(*)[16]>(&rb[0][0]));
+    } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (8 * u < cnt) {
+                tmem_ld_16x256b_x1(taddr + uint32_t(8 * u), ra[u]);
+                tmem_ld_16x256b_x1(taddr + (16u << 16) + uint32_t(8 * u), rb[u]);
+            }
+    }
+    tmem_wait_ld();
+}
+
 // v = hi + lo for two fp32 values: hi = v truncated to bf16 (its top 16 bits),
 // lo = v - hi (exact in fp32) rounded to bf16.  Returns both pairs packed,
 // first value in the low half.
@@ -99,12 +120,14 @@ constexpr int R1 = 64;                                     // rows (t, a) per ti
 constexpr int XT = R1 * KCH * 2;                           // 8 KB: one x tile [64][64]
 constexpr int S1_THREADS = 640;
 constexpr int S1_NX = 4;                                   // loaded x stages
-constexpr int S1_NS = 2;                                   // hi/lo stages
-constexpr int SBOX = RT * 16 * 2;                          // 4 KB: one store box [128 j][16 a]
-constexpr int SG = 4 * SBOX;                               // 16 KB: hi and lo boxes of 32 rows
-constexpr int S1_OFF_S = S1_NX * XT;                       // 32 KB
-constexpr int S1_OFF_STG = S1_OFF_S + S1_NS * 2 * XT;      // 64 KB: two staging buffers per epilogue warpgroup
-constexpr int S1_OFF_BAR = S1_OFF_STG + 4 * SG;            // 128 KB
+constexpr int S1_NS = 4;                                   // hi/lo stages
+constexpr int SBOX = 32 * 16 * 2;                          // 1 KB: one store box [32 j][16 a]
+constexpr int SG = 4 * SBOX;                               // 4 KB: a warp's hi and lo boxes of 32 rows
+constexpr int CT = R1 * KCH * 4;                           // 16 KB: the cinv tile of an x tile [64][64] fp32
+constexpr int S1_OFF_C = S1_NX * XT;                       // 32 KB: cinv stages
+constexpr int S1_OFF_S = S1_OFF_C + S1_NX * CT;            // 96 KB
+constexpr int S1_OFF_STG = S1_OFF_S + S1_NS * 2 * XT;      // 160 KB: two staging buffers per epilogue warp
+constexpr int S1_OFF_BAR = S1_OFF_STG + 8 * 2 * SG;        // 224 KB
 constexpr int B1_XFULL = 0, B1_XEMPTY = S1_NX, B1_SFULL = 2 * S1_NX, B1_SEMPTY = 2 * S1_NX + S1_NS,
               B1_DFULL = 2 * S1_NX + 2 * S1_NS, B1_DEMPTY = B1_DFULL + 2, B1_DONE = B1_DEMPTY + 2,
               B1_COUNT = B1_DONE + 1;
@@ -116,9 +139,9 @@ static_assert(S1_SMEM <= 227 * 1024, "shared memory budget");
 
 template <bool SCALED>
 __global__ void __launch_bounds__(S1_THREADS, 1)
-    kq_two_stage_s1_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_shi,
-                           const __grid_constant__ CUtensorMap tmap_slo, const uint16_t *__restrict__ P2,
-                           const float *__restrict__ cinv, int64_t T, int n1, int n2, unsigned int *err) {
+    kq_two_stage_s1_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_c,
+                           const __grid_constant__ CUtensorMap tmap_shi, const __grid_constant__ CUtensorMap tmap_slo,
+                           const uint16_t *__restrict__ P2, int64_t T, int n1, int n2, unsigned int *err) {
     extern __shared__ __align__(1024) unsigned char s1_raw[];
     const uint32_t raw_addr = smem_u32(s1_raw);
     const uint32_t sbase = align1024(raw_addr);
@@ -151,6 +174,7 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
     }
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&tmap_x);
+        if (SCALED) prefetch_tensormap(&tmap_c);
         prefetch_tensormap(&tmap_shi);
         prefetch_tensormap(&tmap_slo);
     }
@@ -191,6 +215,8 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
 
     if (warp == 0) {
         // ---------------- TMA producer: x tiles [64 rows (t, a)] x [64 b] ----------------
+        // (and with cinv its [64 a] x [64 b] tile, as four 16-row boxes: 16
+        // consecutive rows stay in one token since n1 is a multiple of 16)
         Ring r;
         int issued = 0;
         bool ok = true;
@@ -200,8 +226,14 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
                                                               kSiteTwoStage, kWaitLimitNs, false, err));
                 if (!ok) break;
                 if (elect_one()) {
-                    mbar_arrive_expect_tx(bar(B1_XFULL + r.idx), XT);
+                    mbar_arrive_expect_tx(bar(B1_XFULL + r.idx), SCALED ? XT + CT : XT);
                     tma_load_2d(sbase + uint32_t(r.idx * XT), &tmap_x, kc * KCH, tile * R1, bar(B1_XFULL + r.idx));
+                    if (SCALED) {
+#pragma unroll
+                        for (int b = 0; b < 4; ++b)
+                            tma_load_2d(sbase + uint32_t(S1_OFF_C + r.idx * CT + b * (CT / 4)), &tmap_c, kc * KCH,
+                                        (tile * R1 + 16 * b) % n1, bar(B1_XFULL + r.idx));
+                    }
                 }
                 __syncwarp();
                 ++issued;
@@ -258,89 +290,68 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
     } else if (SCALED && warp >= 4 && warp < 12) {
         // ---------------- x' = x o cinv split into hi/lo bf16 tiles ----------------
         // Thread xt takes 16-byte chunk c = xt % 8 (8 values of b) of rows
-        // xt / 8 and xt / 8 + 32; the swizzled offset is the same in every tile.
-        // cinv for the next chunk is loaded while this one is split.
+        // xt / 8 and xt / 8 + 32; the swizzled offset is the same in every tile,
+        // and the matching cinv values sit at row r, bytes [32 c, 32 c + 32) of
+        // the stage's cinv tile.
         const int xt = tid - 128;
         const int c = xt & 7;
-        auto load_cinv = [&](int tile, int kc, float4 (&cv)[2][2]) {
-            const int b = kc * KCH + 8 * c;
+        Ring rx, rs;
+        for (int tile = first; tile < ntiles; tile += stride) {
+            bool ok = true;
+            for (int kc = 0; kc < KC; ++kc, rx.next(S1_NX), rs.next(S1_NS)) {
+                ok = wait_bounded_err(bar(B1_XFULL + rx.idx), rx.phase, s_abort, kSiteTwoStage, kWaitLimitNs, false,
+                                      err);
+                ok = ok && wait_bounded_err(bar(B1_SEMPTY + rs.idx), rs.phase ^ 1u, s_abort, kSiteTwoStage,
+                                            kWaitLimitNs, false, err);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                const unsigned char *src = smem + rx.idx * XT;
+                const unsigned char *csrc = smem + S1_OFF_C + rx.idx * CT;
+                unsigned char *dhi = smem + S1_OFF_S + rs.idx * 2 * XT;
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                if (tile < ntiles && b < n2) {  // chunks past n2 hold zeros from the load
-                    const int a = (tile * R1 + (xt >> 3) + 32 * i) % n1;
-                    const float4 *cp = reinterpret_cast<const float4 *>(cinv + a * n2 + b);
-                    cv[i][0] = __ldg(cp);
-                    cv[i][1] = __ldg(cp + 1);
-                } else {
-                    cv[i][0] = cv[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int i = 0; i < 2; ++i) {
+                    const int r = (xt >> 3) + 32 * i;
+                    const uint32_t off = uint32_t(r * 128 + ((c ^ (r & 7)) << 4));
+                    const uint4 v = *reinterpret_cast<const uint4 *>(src + off);
+                    const float4 c0 = *reinterpret_cast<const float4 *>(csrc + r * 256 + 32 * c);
+                    const float4 c1 = *reinterpret_cast<const float4 *>(csrc + r * 256 + 32 * c + 16);
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                    const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                    uint32_t h[4], l[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        hi_lo_pair(__uint_as_float(w[e] << 16) * cs[2 * e],
+                                   __uint_as_float(w[e] & 0xFFFF0000u) * cs[2 * e + 1], h[e], l[e]);
+                    *reinterpret_cast<uint4 *>(dhi + off) = make_uint4(h[0], h[1], h[2], h[3]);
+                    *reinterpret_cast<uint4 *>(dhi + XT + off) = make_uint4(l[0], l[1], l[2], l[3]);
+                }
+                fence_proxy_async_smem();  // tiles visible to the tensor cores
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(bar(B1_XEMPTY + rx.idx));
+                    mbar_arrive(bar(B1_SFULL + rs.idx));
                 }
             }
-        };
-        Ring rx, rs;
-        float4 cur[2][2], nxt[2][2];
-        int tile = first, kc = 0;
-        load_cinv(tile, kc, cur);
-        while (tile < ntiles) {
-            int ntile = tile, nkc = kc + 1;
-            if (nkc == KC) {
-                nkc = 0;
-                ntile += stride;
-            }
-            load_cinv(ntile, nkc, nxt);
-            bool ok = wait_bounded_err(bar(B1_XFULL + rx.idx), rx.phase, s_abort, kSiteTwoStage, kWaitLimitNs, false,
-                                       err);
-            ok = ok && wait_bounded_err(bar(B1_SEMPTY + rs.idx), rs.phase ^ 1u, s_abort, kSiteTwoStage,
-                                        kWaitLimitNs, false, err);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            const unsigned char *src = smem + rx.idx * XT;
-            unsigned char *dhi = smem + S1_OFF_S + rs.idx * 2 * XT;
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int r = (xt >> 3) + 32 * i;
-                const uint32_t off = uint32_t(r * 128 + ((c ^ (r & 7)) << 4));
-                const uint4 v = *reinterpret_cast<const uint4 *>(src + off);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                const float cs[8] = {cur[i][0].x, cur[i][0].y, cur[i][0].z, cur[i][0].w,
-                                     cur[i][1].x, cur[i][1].y, cur[i][1].z, cur[i][1].w};
-                uint32_t h[4], l[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    hi_lo_pair(__uint_as_float(w[e] << 16) * cs[2 * e],
-                               __uint_as_float(w[e] & 0xFFFF0000u) * cs[2 * e + 1], h[e], l[e]);
-                *reinterpret_cast<uint4 *>(dhi + off) = make_uint4(h[0], h[1], h[2], h[3]);
-                *reinterpret_cast<uint4 *>(dhi + XT + off) = make_uint4(l[0], l[1], l[2], l[3]);
-            }
-            fence_proxy_async_smem();  // tiles visible to the tensor cores
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar(B1_XEMPTY + rx.idx));
-                mbar_arrive(bar(B1_SFULL + rs.idx));
-            }
-            rx.next(S1_NX);
-            rs.next(S1_NS);
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                cur[i][0] = nxt[i][0];
-                cur[i][1] = nxt[i][1];
-            }
-            tile = ntile;
-            kc = nkc;
+            if (!ok) break;
         }
     } else if (warp >= 12) {
         // ---------------- epilogue: D1 -> Z^T hi/lo boxes -> TMA stores ----------------
-        // Thread = TMEM lane = j (within a slice).  Each 32-row half of a slice's
-        // accumulator becomes two [128 j][16 a] boxes of hi and two of lo (16
-        // consecutive rows stay in one token since n1 is a multiple of 16),
-        // staged in shared memory (two buffers) and stored by one thread.
-        const int ew = (warp - 12) >> 2, q = warp & 3, et = tid - 384 - 128 * ew;
-        const int j = 32 * q + lane;
-        const uint32_t nb_leave = 1u + uint32_t(ew), nb_stage = 3u + uint32_t(ew);
+        // Thread = TMEM lane = row m of a slice.  Each warp turns its 32 lanes of a
+        // 32-row half of the accumulator into two [32 m][16 a] boxes of hi and
+        // two of lo (16 consecutive rows stay in one token since n1 is a
+        // multiple of 16), staged in its own two shared buffers and stored by
+        // its own TMA stores: no barrier between warps.  Warpgroups 12-15 and
+        // 16-19 take alternate halves.
+        const int ew = (warp - 12) >> 2, q = warp & 3;
+        unsigned char *wstg = smem + S1_OFF_STG + (warp - 12) * 2 * SG;
+        const uint32_t wsa = sbase + uint32_t(S1_OFF_STG + (warp - 12) * 2 * SG);
+        const int sw = (lane >> 2) & 1;  // chunk order that spreads the 16-byte stores over all banks
         Ring rd;
         int sb = 0;
         for (int tile = first; tile < ntiles; tile += stride, rd.next(2)) {
             const bool ok = wait_bounded_err(bar(B1_DFULL + rd.idx), rd.phase, s_abort, kSiteTwoStage, kWaitLimitNs,
                                              false, err);
-            if (named_barrier_any(nb_leave, 128, !__all_sync(0xffffffffu, ok))) break;  // leave together
+            if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             for (int s = 0; s < J; ++s)
                 for (int hf = ew; hf < 2; hf += 2) {
@@ -358,17 +369,16 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         hi_lo_pair(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]), h[e], l[e]);
-                    if (et == 0) bulk_wait_read<1>();  // the stores that used this buffer have read it
-                    named_barrier_sync(nb_stage, 128);
-                    unsigned char *stg = smem + S1_OFF_STG + (2 * ew + sb) * SG;
-                    const int sw = (j >> 2) & 1;  // chunk order that spreads the 16-byte stores over all banks
+                    if (lane == 0) bulk_wait_read<1>();  // the stores that used this buffer have read it
+                    __syncwarp();
+                    unsigned char *stg = wstg + sb * SG;
 #pragma unroll
                     for (int bx = 0; bx < 2; ++bx) {
                         const uint4 h0 = make_uint4(h[8 * bx], h[8 * bx + 1], h[8 * bx + 2], h[8 * bx + 3]);
                         const uint4 h1 = make_uint4(h[8 * bx + 4], h[8 * bx + 5], h[8 * bx + 6], h[8 * bx + 7]);
                         const uint4 l0 = make_uint4(l[8 * bx], l[8 * bx + 1], l[8 * bx + 2], l[8 * bx + 3]);
                         const uint4 l1 = make_uint4(l[8 * bx + 4], l[8 * bx + 5], l[8 * bx + 6], l[8 * bx + 7]);
-                        const uint32_t off = uint32_t(bx * SBOX + j * 32);
+                        const uint32_t off = uint32_t(bx * SBOX + lane * 32);
                         const uint32_t o_first = sw ? 16u : 0u, o_second = sw ? 0u : 16u;
                         *reinterpret_cast<uint4 *>(stg + off + o_first) = sw ? h1 : h0;
                         *reinterpret_cast<uint4 *>(stg + 2 * SBOX + off + o_first) = sw ? l1 : l0;
@@ -376,15 +386,15 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
                         *reinterpret_cast<uint4 *>(stg + 2 * SBOX + off + o_second) = sw ? l0 : l1;
                     }
                     fence_proxy_async_smem();  // staging visible to the tensor stores
-                    named_barrier_sync(nb_stage, 128);
-                    if (et == 0) {
-                        const uint32_t sa = sbase + uint32_t(S1_OFF_STG + (2 * ew + sb) * SG);
+                    __syncwarp();
+                    if (lane == 0) {
+                        const uint32_t sa = wsa + uint32_t(sb * SG);
 #pragma unroll
                         for (int bx = 0; bx < 2; ++bx) {
                             const int R = tile * R1 + 32 * hf + 16 * bx;
                             if (R < rows) {
                                 const int t = R / n1, a0 = R - t * n1;
-                                const int y = t * Jp + RT * s;
+                                const int y = t * Jp + RT * s + 32 * q;
                                 tma_store_2d(&tmap_shi, a0, y, sa + uint32_t(bx * SBOX));
                                 tma_store_2d(&tmap_slo, a0, y, sa + uint32_t(2 * SBOX + bx * SBOX));
                             }
@@ -394,7 +404,7 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
                     sb ^= 1;
                 }
         }
-        if (et == 0) bulk_wait<0>();
+        if (lane == 0) bulk_wait<0>();
     }
 
     tc_fence_before();
@@ -417,7 +427,7 @@ constexpr int S2_SMEM_MAX = 227 * 1024;
 // from the 1024-aligned base) and its barrier indices.
 struct S2Layout {
     int n1, n2, J, AC, NA, NB, dcols;
-    int off_b2, off_a, off_stg, off_bar, off_red, off_misc, smem;
+    int off_b2, off_a, off_bar, off_red, off_misc, smem;
     __host__ __device__ int AFULL(int s) const { return s; }
     __host__ __device__ int AEMPTY(int s) const { return NA + s; }
     __host__ __device__ int DFULL(int b, int s) const { return 2 * NA + b * J + s; }
@@ -437,12 +447,10 @@ __host__ __device__ inline S2Layout s2_layout(int n1, int n2) {
     L.off_b2 = 0;
     const int b2 = L.AC * n1 * 128;                 // P1^T chunks [n1 rows][128 B]
     L.off_a = (b2 + 1023) & ~1023;
-    const int stg = n1 * n2 / 2;                    // one token's codes
-    const int fixed = 1024 /* alignment slack */ + L.off_a + stg + 8 * (2 * S2_MAX_NA + 9) + 64 + 16;
+    const int fixed = 1024 /* alignment slack */ + L.off_a + 8 * (2 * S2_MAX_NA + 9) + 64 + 16;
     const int na = (S2_SMEM_MAX - fixed) / (2 * TILE);
     L.NA = na > S2_MAX_NA ? S2_MAX_NA : na;
-    L.off_stg = L.off_a + L.NA * 2 * TILE;
-    L.off_bar = (L.off_stg + stg + 7) & ~7;
+    L.off_bar = L.off_a + L.NA * 2 * TILE;
     L.off_red = L.off_bar + 8 * L.nbar();
     L.off_misc = L.off_red + 64;                    // 2 x 8 floats
     L.smem = L.off_misc + 16 + 1024;
@@ -584,7 +592,6 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
         const int h = n1 / 2;
         const int one = *reinterpret_cast<volatile int *>(smem + L.off_misc + 8);
         float *red = reinterpret_cast<float *>(smem + L.off_red);
-        unsigned char *stg = smem + L.off_stg;
         Ring rd;
         int par = 0;
         for (int64_t t = blockIdx.x; t < T; t += gridDim.x, rd.next(L.NB), par ^= 1) {
@@ -604,13 +611,7 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
                 for (int c = 0; c < h; c += 32) {
                     const int cnt = h - c < 32 ? h - c : 32;  // a multiple of 8
                     uint32_t ra[4][4], rb[4][4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        if (8 * u < cnt) {
-                            tmem_ld_16x256b_x1(lanes + uint32_t(s * n1 + c + 8 * u), ra[u]);
-                            tmem_ld_16x256b_x1(lanes + (16u << 16) + uint32_t(s * n1 + c + 8 * u), rb[u]);
-                        }
-                    tmem_wait_ld();
+                    load_run(lanes + uint32_t(s * n1 + c), cnt, ra, rb);
                     if (valid) {
 #pragma unroll
                         for (int u = 0; u < 4; ++u)
@@ -624,7 +625,6 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
             }
             const unsigned mw = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
             if (lane == 0) red[8 * par + (warp - 4)] = __uint_as_float(mw);
-            if (et == 0) bulk_wait_read<0>();  // the previous token's codes have left the staging buffer
             if (named_barrier_any(1, 256, !ok)) break;  // all epilogue warps leave together
             float M = red[8 * par];
 #pragma unroll
@@ -632,20 +632,17 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
             const float sc = alpha * M * (1.0f / 7.0f);
             const float inv = sc > 0.0f ? fminf(__fdividef(1.0f, sc), 3.0e38f) : 0.0f;
             if (et == 0) scale_out[t] = sc;
-            // pass 2: codes, two bytes (columns 4 g .. 4 g + 3) per row i
+            // pass 2: codes, two bytes (columns 4 g .. 4 g + 3) per row i, stored
+            // straight to the token's row of q_out (the eight groups g of a warp
+            // fill 16 contiguous bytes of each row)
+            uint8_t *qt = q_out + t * (n / 2);
             for (int s = 0; s < L.J; ++s) {
                 const int jb = RT * s + 32 * q + 4 * g;
                 const bool store = jb < n2;
                 for (int c = 0; c < h; c += 32) {
                     const int cnt = h - c < 32 ? h - c : 32;
                     uint32_t ra[4][4], rb[4][4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        if (8 * u < cnt) {
-                            tmem_ld_16x256b_x1(lanes + uint32_t(s * n1 + c + 8 * u), ra[u]);
-                            tmem_ld_16x256b_x1(lanes + (16u << 16) + uint32_t(s * n1 + c + 8 * u), rb[u]);
-                        }
-                    tmem_wait_ld();
+                    load_run(lanes + uint32_t(s * n1 + c), cnt, ra, rb);
                     if (c + 32 >= h) {  // this warp's last read of the slice
                         tc_fence_before();
                         __syncwarp();
@@ -662,20 +659,13 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
                                                              round_code_ts(ra[u][d], inv, one), hi);
                                 if (store) {
                                     const int i = ew * h + c + 8 * u + 2 * cp + d;
-                                    *reinterpret_cast<uint16_t *>(stg + ((i * n2 + jb) >> 1)) = uint16_t(w);
+                                    *reinterpret_cast<uint16_t *>(qt + ((i * n2 + jb) >> 1)) = uint16_t(w);
                                 }
                             }
                         }
                 }
             }
-            fence_proxy_async_smem();  // staging writes visible to the bulk copy
-            named_barrier_sync(2, 256);
-            if (et == 0) {
-                bulk_store(q_out + t * (n / 2), sbase + uint32_t(L.off_stg), uint32_t(n / 2));
-                bulk_commit();
-            }
         }
-        if (et == 0) bulk_wait<0>();
     }
 
     tc_fence_before();
@@ -737,24 +727,38 @@ cudaError_t launch_two_stage(const LaunchArgs &a, void *workspace) {
     const uint64_t zrows = uint64_t(a.T) * uint64_t(RT * slices(a.n2));  // Z^T rows, padded per token
     uint16_t *zhi = static_cast<uint16_t *>(workspace);
     uint16_t *zlo = zhi + zrows * uint64_t(a.n1);
-    CUtensorMap tx, shi, slo, lhi, llo;
+    CUtensorMap tx, tc, shi, slo, lhi, llo;
     if (encode_bf16_2d(&tx, a.x, uint64_t(a.n2), uint64_t(a.T) * a.n1, KCH, R1, CU_TENSOR_MAP_SWIZZLE_128B) !=
             CUDA_SUCCESS ||
-        encode_bf16_2d(&shi, zhi, uint64_t(a.n1), zrows, 16, RT, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
-        encode_bf16_2d(&slo, zlo, uint64_t(a.n1), zrows, 16, RT, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
+        encode_bf16_2d(&shi, zhi, uint64_t(a.n1), zrows, 16, 32, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
+        encode_bf16_2d(&slo, zlo, uint64_t(a.n1), zrows, 16, 32, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
         encode_bf16_2d(&lhi, zhi, uint64_t(a.n1), zrows, KCH, RT, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
         encode_bf16_2d(&llo, zlo, uint64_t(a.n1), zrows, KCH, RT, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+    if (a.cinv) {
+        // cinv as [n1 rows][n2 cols] fp32; boxes [16 rows][64 cols], columns past n2 read as zero
+        PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+        const cuuint64_t dims[2] = {cuuint64_t(a.n2), cuuint64_t(a.n1)};
+        const cuuint64_t stride[1] = {cuuint64_t(a.n2) * 4};
+        const cuuint32_t box[2] = {cuuint32_t(KCH), 16u};
+        const cuuint32_t estr[2] = {1u, 1u};
+        if (!encode || encode(&tc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(a.cinv), dims, stride, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    } else {
+        tc = tx;  // unused without cinv
+    }
 
     // stage 1: persistent CTAs over 64-row tiles
     const int64_t ntiles = (a.T * a.n1 + R1 - 1) / R1;
     const int64_t g1 = ntiles < a.num_sms ? ntiles : a.num_sms;
     if (a.cinv)
-        kq_two_stage_s1_kernel<true><<<unsigned(g1), S1_THREADS, S1_SMEM, a.stream>>>(tx, shi, slo, a.P2, a.cinv, a.T,
-                                                                                      a.n1, a.n2, err);
+        kq_two_stage_s1_kernel<true><<<unsigned(g1), S1_THREADS, S1_SMEM, a.stream>>>(tx, tc, shi, slo, a.P2, a.T, a.n1,
+                                                                                      a.n2, err);
     else
-        kq_two_stage_s1_kernel<false><<<unsigned(g1), S1_THREADS, S1_SMEM, a.stream>>>(tx, shi, slo, a.P2, nullptr,
-                                                                                       a.T, a.n1, a.n2, err);
+        kq_two_stage_s1_kernel<false><<<unsigned(g1), S1_THREADS, S1_SMEM, a.stream>>>(tx, tc, shi, slo, a.P2, a.T,
+                                                                                       a.n1, a.n2, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
