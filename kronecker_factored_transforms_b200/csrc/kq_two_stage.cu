@@ -136,6 +136,7 @@ constexpr int S1_SMEM = S1_OFF_MISC + 16 + 1024;           // + slack for 1024-b
 constexpr uint32_t S1_TMEM_COLS = 512;
 constexpr uint32_t S1_DCOL = 256;                          // A1 slices at 0 and 128; D1 [2 buffers][2 slices][64]
 static_assert(S1_SMEM <= 227 * 1024, "shared memory budget");
+static_assert(S1_OFF_BAR >= kMaxFactor * kMaxFactor * 2, "P2 staging at start fits before the barriers");
 
 template <bool SCALED>
 __global__ void __launch_bounds__(S1_THREADS, 1)
@@ -187,11 +188,31 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + S1_OFF_MISC);
 
+    // P2 into shared memory first (row-major, the pipeline buffers are not in
+    // use yet): 16-byte loads, eight per thread in flight.
+    {
+        const int units = n2 * n2 / 8;
+        for (int u0 = tid; u0 < units; u0 += 8 * S1_THREADS) {
+            uint4 v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int u = u0 + q * S1_THREADS;
+                if (u < units) v[q] = __ldg(reinterpret_cast<const uint4 *>(P2) + u);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int u = u0 + q * S1_THREADS;
+                if (u < units) *reinterpret_cast<uint4 *>(smem + 16 * u) = v[q];
+            }
+        }
+    }
+    __syncthreads();
     if (warp >= 12) {
         // A1 = P2^T into TMEM: slice s at columns [128 s, 128 s + 32 KC); lane m
         // holds row j = 128 s + lane_column(m), K pairs (b, b + 1) packed per
         // column; zero outside n2 (rows j >= n2 give zero accumulators).
         // Warpgroup 12-15 writes slice 0, 16-19 slice 1.
+        const uint16_t *P2s = reinterpret_cast<const uint16_t *>(smem);
         const uint32_t lanes = tmem + (uint32_t(32 * (warp & 3)) << 16);
         for (int s = (warp - 12) >> 2; s < J; s += 2) {
             const int jg = RT * s + tile::lane_column(32 * (warp & 3) + lane);
@@ -200,8 +221,8 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int b = 32 * c16 + 2 * e;
-                    const uint32_t v0 = (jg < n2 && b < n2) ? P2[b * n2 + jg] : 0u;
-                    const uint32_t v1 = (jg < n2 && b + 1 < n2) ? P2[(b + 1) * n2 + jg] : 0u;
+                    const uint32_t v0 = (jg < n2 && b < n2) ? P2s[b * n2 + jg] : 0u;
+                    const uint32_t v1 = (jg < n2 && b + 1 < n2) ? P2s[(b + 1) * n2 + jg] : 0u;
                     w[e] = v0 | (v1 << 16);
                 }
                 tmem_st_32x32b_x16(lanes + uint32_t(RT * s + 16 * c16), w);
@@ -209,6 +230,7 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
         }
         tmem_wait_st();
     }
+    fence_proxy_async_smem();  // the staged P2 is read before TMA writes reuse the buffers
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -495,12 +517,37 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
         tmem_relinquish();
     }
     // B2 = P1^T in 128B-swizzled K-major chunks: row i, K = a; zero for a >= n1.
-    for (int idx = tid; idx < L.AC * KCH * n1; idx += S2_THREADS) {
-        const int a = idx / n1, i = idx - a * n1;
-        const uint16_t v = a < n1 ? P1[a * n1 + i] : uint16_t(0);
-        const int k = a & (KCH - 1);
-        *reinterpret_cast<uint16_t *>(smem + L.off_b2 + (a >> 6) * n1 * 128 + i * 128 +
-                                      ((((k >> 3) ^ (i & 7)) << 4) | ((k & 7) << 1))) = v;
+    // A unit is one row i and eight consecutive a: eight loads (consecutive
+    // threads take consecutive i, so each load is coalesced), one 16-byte store
+    // (the swizzle spreads consecutive rows over all banks); four units in
+    // flight per thread.
+    {
+        const int units = L.AC * KCH / 8 * n1;
+        for (int u0 = tid; u0 < units; u0 += 4 * S2_THREADS) {
+            uint32_t w[4][4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int u = u0 + q * S2_THREADS;
+                const int i = u % n1, a0 = 8 * (u / n1);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int a = a0 + 2 * e;
+                    const uint32_t lo = (u < units && a < n1) ? P1[a * n1 + i] : 0u;
+                    const uint32_t hi = (u < units && a + 1 < n1) ? P1[(a + 1) * n1 + i] : 0u;
+                    w[q][e] = lo | (hi << 16);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int u = u0 + q * S2_THREADS;
+                if (u < units) {
+                    const int i = u % n1, a0 = 8 * (u / n1);
+                    *reinterpret_cast<uint4 *>(smem + L.off_b2 + (a0 >> 6) * n1 * 128 + i * 128 +
+                                               ((((a0 & 63) >> 3) ^ (i & 7)) << 4)) =
+                        make_uint4(w[q][0], w[q][1], w[q][2], w[q][3]);
+                }
+            }
+        }
     }
     fence_proxy_async_smem();
     tc_fence_before();
