@@ -265,32 +265,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         constexpr int kSetupThreads = 15 * 32;
         const int st = 32 * setup_idx + lane;
         // B2[i][a] = P1[a][i] (rows i, K = a), 128B-swizzled K-major, zero beyond a = n1.
-        // Each thread reads whole 16-byte pieces of rows of P1 (all its loads first)
-        // and scatters their eight values down a column of B2.
         {
-            constexpr int PIECES = N1 * N1 / 8, PER = (PIECES + kSetupThreads - 1) / kSetupThreads;
-            uint4 v[PER];
+            // A piece is one row i and eight consecutive a (zero past n1): eight
+            // loads (consecutive threads take consecutive i, so each is
+            // coalesced) and one 16-byte store (the swizzle spreads consecutive
+            // rows over all banks).
+            constexpr int PIECES = C::NCH2 * 8 * N1, PER = (PIECES + kSetupThreads - 1) / kSetupThreads;
+            uint32_t w[PER][4];
 #pragma unroll
             for (int u = 0; u < PER; ++u) {
                 const int c = st + u * kSetupThreads;
-                if (c < PIECES) v[u] = *reinterpret_cast<const uint4 *>(P1 + 8 * c);
+                const int i = c % N1, a0 = 8 * (c / N1);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int a = a0 + 2 * e;
+                    const uint32_t lo = (c < PIECES && a < N1) ? P1[a * N1 + i] : 0u;
+                    const uint32_t hi = (c < PIECES && a + 1 < N1) ? P1[(a + 1) * N1 + i] : 0u;
+                    w[u][e] = lo | (hi << 16);
+                }
             }
 #pragma unroll
             for (int u = 0; u < PER; ++u) {
                 const int c = st + u * kSetupThreads;
                 if (c < PIECES) {
-                    const int a = (8 * c) / N1, i0 = (8 * c) % N1;
-                    const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                    for (int t = 0; t < 8; ++t)
-                        *reinterpret_cast<uint16_t *>(smem + C::OFF_B2 + (a >> 6) * (N1 * 128) + swz128(i0 + t, a & 63)) =
-                            uint16_t(w[t >> 1] >> (16 * (t & 1)));
+                    const int i = c % N1, a0 = 8 * (c / N1);
+                    *reinterpret_cast<uint4 *>(smem + C::OFF_B2 + (a0 >> 6) * (N1 * 128) + swz128(i, a0 & 63)) =
+                        make_uint4(w[u][0], w[u][1], w[u][2], w[u][3]);
                 }
-            }
-            // zero K padding (a in [n1, 64 NCH2))
-            for (int e = st; e < (C::NCH2 * 64 - N1) * N1; e += kSetupThreads) {
-                const int a = N1 + e / N1, i = e % N1;
-                *reinterpret_cast<uint16_t *>(smem + C::OFF_B2 + (a >> 6) * (N1 * 128) + swz128(i, a & 63)) = 0;
             }
         }
         if (!C::A1_TMEM) {
