@@ -10,11 +10,15 @@
 // The 5th-generation tensor cores have no 4-bit integer kind, so each 128-code
 // K chunk goes: packed tiles by TMA -> eight expander warps widen every code q
 // to the int8 16 q (a mask keeps the high nibble where it is, a shift moves the
-// low one up) -> tcgen05.mma kind::i8 (s8 x s8 -> s32 in TMEM).  Within every
-// 8-code group the expanders write the even codes before the odd ones, the
-// same way for both operands, which leaves every dot product unchanged.  The
-// s32 sums are 256 times the code sums and exact (|sum| <= 16384 K < 2^31); the
-// epilogue shifts the factor out and applies (float(sum) * sx[m]) * sw[o].
+// low one up) -> tcgen05.mma kind::i8 (s8 x s8 -> s32 in TMEM).  The widened
+// activation tile goes straight into TMEM (the MMA's A operand, one row per
+// lane, four K bytes per column), the widened weight tile into shared memory
+// (B), which keeps a third of the widened bytes off the shared-memory pipe.
+// Within every 8-code group the expanders write the even codes before the odd
+// ones, the same way for both operands, which leaves every dot product
+// unchanged.  The s32 sums are 256 times the code sums and exact
+// (|sum| <= 16384 K < 2^31); the epilogue shifts the factor out and applies
+// (float(sum) * sx[m]) * sw[o].
 //
 // One CTA per 128 x 256 output tile.  Warps: 0 TMA producer | 1 TMEM
 // allocator + MMA issuer | 4-11 expanders, then the epilogue | 2-3 idle.
@@ -33,18 +37,20 @@ using namespace tc;
 
 constexpr int TM = 128, TN = 256, KC = 128;            // tile rows, columns, codes per K chunk
 constexpr int PA = TM * KC / 2, PB = TN * KC / 2;       // packed bytes per chunk: 8 KB, 16 KB
-constexpr int EA = TM * KC, EB = TN * KC;               // widened int8 bytes per chunk: 16 KB, 32 KB
-constexpr int NS = 4, NE = 2;                           // packed stages, widened stages
+constexpr int EB = TN * KC;                             // widened int8 weight bytes per chunk: 32 KB
+constexpr int NS = 4, NE = 3;                           // packed stages, widened stages
 constexpr int G_THREADS = 384;                          // 12 warps
 constexpr int XW0 = 4, NXW = 8;                         // expander / epilogue warps 4-11
-constexpr int OFF_E = NS * (PA + PB);                   // 96 KB: widened stages (1024-aligned)
-constexpr int OFF_BAR = OFF_E + NE * (EA + EB);
+constexpr int OFF_E = NS * (PA + PB);                   // 96 KB: widened weight stages (1024-aligned)
+constexpr int OFF_BAR = OFF_E + NE * EB;
 constexpr int FULL = 0, EMPTY = NS, XFULL = 2 * NS, XEMPTY = 2 * NS + NE, DONE = 2 * NS + 2 * NE;
 constexpr int NBAR = DONE + 1;
 constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;            // TMEM base, abort flag
 constexpr int G_SMEM = OFF_MISC + 16 + 1024;            // + slack for 1024-byte alignment
-constexpr uint32_t TMEM_COLS = TN;                      // s32 accumulator: 256 columns
-static_assert(OFF_E % 1024 == 0 && (EA + EB) % 1024 == 0 && EA % 1024 == 0, "swizzle atoms");
+constexpr uint32_t TMEM_COLS = 512;                     // s32 accumulator [0, 256) + widened activations
+constexpr uint32_t ACOL = TN;                           // widened activation stage e at columns 256 + 32 e
+static_assert(ACOL + NE * (KC / 4) <= TMEM_COLS, "TMEM budget");
+static_assert(OFF_E % 1024 == 0 && EB % 1024 == 0 && (PA + PB) % 1024 == 0, "swizzle atoms");
 static_assert(G_SMEM <= 227 * 1024, "shared memory budget");
 
 enum : unsigned { kSiteGemm = 64u };
@@ -58,15 +64,15 @@ __host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
            | (uint32_t(M >> 4) << 24);    // M / 16
 }
 
-// D (+)= A B^T with both operands in shared memory, described by the low
-// halves of their 128B-swizzle descriptors.
+// D (+)= A B^T with A in TMEM and B in shared memory, described by the low
+// half of its 128B-swizzle descriptor.
 template <int ACC>
-__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc) {
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\tmov.b64 ad, {%1, %3};\n\tmov.b64 bd, {%2, %3};\n\t"
+        "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\tmov.b64 bd, {%2, %3};\n\t"
         "setp.ne.b32 p, %5, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], ad, bd, %4, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_lo), "r"(b_lo), "r"(kSdescSw128Hi), "r"(idesc), "n"(ACC)
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(kSdescSw128Hi), "r"(idesc), "n"(ACC)
         : "memory");
 }
 
@@ -145,15 +151,15 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                                              err);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            const uint32_t ea = sbase + uint32_t(OFF_E + r.idx * (EA + EB));
-            const uint32_t al = sdesc_sw128_lo(ea), bl = sdesc_sw128_lo(ea + EA);
+            const uint32_t bl = sdesc_sw128_lo(sbase + uint32_t(OFF_E + r.idx * EB));
+            const uint32_t at = tmem + ACOL + uint32_t(r.idx * (KC / 4));
             if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < KC / 32; ++kk) {  // K = 32 int8 per MMA: +32 bytes
+                for (int kk = 0; kk < KC / 32; ++kk) {  // K = 32 int8 per MMA: 8 TMEM columns, +32 bytes of B
                     if ((kt | kk) != 0)
-                        mma_i8<1>(tmem, al + 2 * kk, bl + 2 * kk, idesc);
+                        mma_i8_ts<1>(tmem, at + 8 * kk, bl + 2 * kk, idesc);
                     else
-                        mma_i8<0>(tmem, al + 2 * kk, bl + 2 * kk, idesc);
+                        mma_i8_ts<0>(tmem, at + 8 * kk, bl + 2 * kk, idesc);
                 }
                 tc_commit(bar(XEMPTY + r.idx));  // widened stage free once these MMAs complete
             }
@@ -165,11 +171,19 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         wait_bounded_err(bar(DONE), 0u, s_abort, kSiteGemm, kWaitLimitNs, true, err);
         __syncwarp();
     } else if (warp >= XW0 && warp < XW0 + NXW) {
-        // ---------------- expanders: packed INT4 -> int8 (x16), swizzled K-major ----------------
+        // ---------------- expanders: packed INT4 -> int8 (x16) ----------------
+        // Activations: thread (warp w, lane) widens half (hh = (w - 4) / 4) of
+        // row m = 32 (w % 4) + lane: two 16-byte units of the packed tile (64B
+        // swizzle: unit c of row m at m * 64 + 16 (c ^ ((m >> 1) & 3)), so the
+        // eight rows of a shared-memory phase hit eight bank groups) become
+        // sixteen TMEM columns of lane m.  Weights: four 16-byte units per thread
+        // into the 128B-swizzled K-major shared tile.
         const int xt = tid - XW0 * 32;                // 0 .. 255
-        constexpr int UNITS = (TM + TN) * (KC / 32);  // 16-byte packed units per chunk: 1536
-        constexpr int UPT = UNITS / (NXW * 32);       // 6 per thread
-        static_assert(UNITS % (NXW * 32) == 0, "unit split");
+        const int hh = (warp - XW0) >> 2, qa = warp & 3;
+        const int am = 32 * qa + lane;                // activation row = TMEM lane
+        constexpr int UB = TN * (KC / 32);            // 16-byte packed weight units per chunk: 1024
+        constexpr int UPB = UB / (NXW * 32);          // 4 per thread
+        static_assert(UB % (NXW * 32) == 0, "unit split");
         Ring rs, re;
         bool ok = true;
         for (int kt = 0; kt < KT; ++kt, rs.next(NS), re.next(NE)) {
@@ -177,32 +191,48 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             ok = ok && wait_bounded_err(bar(XEMPTY + re.idx), re.phase ^ 1u, s_abort, kSiteGemm, kWaitLimitNs,
                                         false, err);
             if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
             const unsigned char *pk = smem + rs.idx * (PA + PB);
-            unsigned char *ex = smem + OFF_E + re.idx * (EA + EB);
-            uint4 v[UPT];
+            unsigned char *ex = smem + OFF_E + re.idx * EB;
+            uint4 va[2], vb[UPB];
 #pragma unroll
-            for (int i = 0; i < UPT; ++i) {
-                const int u = xt + i * NXW * 32;  // A units first (row u / 4), then B
-                v[i] = *reinterpret_cast<const uint4 *>(pk + u * 16);
+            for (int c = 0; c < 2; ++c) {
+                const int u = 2 * hh + c;
+                va[c] = *reinterpret_cast<const uint4 *>(pk + am * 64 + ((u ^ ((am >> 1) & 3)) << 4));
             }
 #pragma unroll
-            for (int i = 0; i < UPT; ++i) {
-                const int u = xt + i * NXW * 32;
-                const bool isb = u >= TM * (KC / 32);
-                const int ub = isb ? u - TM * (KC / 32) : u;
-                const int r = ub >> 2, q = ub & 3;  // row, 16-byte unit within the row's 64 packed bytes
-                unsigned char *dst = ex + (isb ? EA : 0);
-                const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-                uint32_t o[8];
+            for (int i = 0; i < UPB; ++i)
+                vb[i] = *reinterpret_cast<const uint4 *>(pk + PA + (xt + i * NXW * 32) * 16);
+            // activations -> TMEM: unit c gives columns 8 c .. 8 c + 7 of this half
+            uint32_t o[16];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const uint32_t w[4] = {va[c].x, va[c].y, va[c].z, va[c].w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    o[2 * j] = (w[j] << 4) & 0xF0F0F0F0u;  // even codes of the 8-code group, x16
-                    o[2 * j + 1] = w[j] & 0xF0F0F0F0u;     // odd codes, x16
+                    o[8 * c + 2 * j] = (w[j] << 4) & 0xF0F0F0F0u;  // even codes of the 8-code group, x16
+                    o[8 * c + 2 * j + 1] = w[j] & 0xF0F0F0F0u;     // odd codes, x16
                 }
-                *reinterpret_cast<uint4 *>(dst + sw128_chunk(r, 2 * q)) = make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4 *>(dst + sw128_chunk(r, 2 * q + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
             }
-            fence_proxy_async_smem();  // widened tile visible to the tensor cores
+            tmem_st_32x32b_x16(tmem + (uint32_t(32 * qa) << 16) + ACOL + uint32_t(re.idx * (KC / 4) + 16 * hh), o);
+            // weights -> shared memory
+#pragma unroll
+            for (int i = 0; i < UPB; ++i) {
+                const int ub = xt + i * NXW * 32;
+                const int r = ub >> 2, q = ub & 3;  // row, 16-byte unit within the row's 64 packed bytes
+                const uint32_t w[4] = {vb[i].x, vb[i].y, vb[i].z, vb[i].w};
+                uint32_t e[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    e[2 * j] = (w[j] << 4) & 0xF0F0F0F0u;
+                    e[2 * j + 1] = w[j] & 0xF0F0F0F0u;
+                }
+                *reinterpret_cast<uint4 *>(ex + sw128_chunk(r, 2 * q)) = make_uint4(e[0], e[1], e[2], e[3]);
+                *reinterpret_cast<uint4 *>(ex + sw128_chunk(r, 2 * q + 1)) = make_uint4(e[4], e[5], e[6], e[7]);
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();  // widened weight tile visible to the tensor cores
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar(EMPTY + rs.idx));  // packed stage read
@@ -279,7 +309,7 @@ cudaError_t launch_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *
     const cuuint32_t boxa[2] = {cuuint32_t(KC / 2), cuuint32_t(TM)}, boxb[2] = {cuuint32_t(KC / 2), cuuint32_t(TN)};
     const cuuint32_t estr[2] = {1u, 1u};
     CUresult r = encode(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(qx), da, stride, boxa, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     r = encode(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(qw), db, stride, boxb, estr,
