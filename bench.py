@@ -54,10 +54,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["transform", "gemm", "two_stage"], default="transform",
+    ap.add_argument("--workload", choices=["transform", "gemm", "two_stage", "headwise"], default="transform",
                     help="transform: the fused transform + INT4 path (default); gemm: the W4A4 product "
                          "of packed codes that consumes it (M = N = K = 8192); two_stage: the path for "
-                         "factors above 128 (--two-stage-config)")
+                         "factors above 128 (--two-stage-config); headwise: the per-head key/value "
+                         "transform + INT4 (8192 tokens x 32 heads x 128)")
     ap.add_argument("--two-stage-config", choices=["square65536", "ffn28672"], default="square65536")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -355,6 +356,64 @@ def run_two_stage(args):
     return 0
 
 
+def run_headwise(args):
+    """The per-head transform of the key/value cache: 8192 tokens x 32 heads of
+    head_dim 128 (262144 rows), one bf16 factor, INT4 per row.  One step is one
+    kq_headwise_transform_quant call; inputs rotate over enough buffer sets to
+    exceed 2x L2.  Roofline: algorithmic bytes 2.5 D + 4 per row at the measured
+    HBM peak (2 D^2 flops per row are far below the tensor peak).  Single GPU."""
+    import torch
+    from kronecker_factored_transforms_b200 import _lib
+    T, heads, D = 8192, 32, 128
+    R = T * heads
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(4096)
+    set_bytes = R * (2 * D + D // 2 + 4)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    nset = max(2, math.ceil(2 * l2 / set_bytes) + 1)
+    xs = [torch.randn((T, heads * D), device=dev, generator=g).to(torch.bfloat16) for _ in range(nset)]
+    Q, _ = torch.linalg.qr(torch.randn((D, D), device=dev, generator=g, dtype=torch.float64))
+    Ph = Q.to(torch.bfloat16).contiguous()
+    qs = [torch.empty((T, heads * D // 2), dtype=torch.uint8, device=dev) for _ in range(nset)]
+    ss = [torch.empty((T, heads), dtype=torch.float32, device=dev) for _ in range(nset)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        _lib.kq_headwise_transform_quant(xs[i % nset], Ph, 0.9, qs[i % nset], ss[i % nset], T, heads, D,
+                                         stream=stream.cuda_stream)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(0)
+    with sampler:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    if _lib.kq_device_error(stream) != 0:
+        raise RuntimeError("a bounded wait timed out inside the kernel")
+    ms = e0.elapsed_time(e1) / args.steps
+    hbm_peak, _, kind = measured_peaks()
+    bytes_launch = R * (2 * D + D // 2 + 4)
+    achieved = bytes_launch / (ms / 1e3) / 1e9
+    line = {"metric": "rows/s and % HBM roofline of the per-head key/value transform + INT4", "value": R / (ms / 1e3),
+            "unit": "rows/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "headwise: %d tokens x %d heads x head_dim %d, N(0,1) rows, orthogonal bf16 "
+                                   "factor, alpha 0.9" % (T, heads, D), "rows": R, "head_dim": D,
+                       "l2": "inputs rotate over %d buffer sets (%.0f MB > 2x L2)" % (nset, nset * set_bytes / 1e6)},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": None, "peak_source": "%s (MEASURED_PEAKS.json)" % kind,
+                         "bytes_per_launch": bytes_launch},
+            "gpu_launches": args.steps, "clocks": sampler.report()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -363,6 +422,8 @@ def main():
         return run_gemm(args)
     if args.workload == "two_stage":
         return run_two_stage(args)
+    if args.workload == "headwise":
+        return run_headwise(args)
 
     import torch
     import torch.distributed as dist
