@@ -133,6 +133,9 @@ def whole_job_tokens_per_s(world, tokens_per_rank, steps, ms):
 # CPU oracle timing (baseline leg and the reference arm).
 
 def time_oracle(w, seconds, max_tokens=None):
+    """The oracle on the host cores for about `seconds`: passes over the
+    workload's rows, in pieces of about a second, until the time is reached
+    (or `max_tokens`).  Returns (tokens/s, threads, tokens, seconds)."""
     import oracle
     oracle.build()
     nth = oracle.default_threads()
@@ -140,22 +143,21 @@ def time_oracle(w, seconds, max_tokens=None):
     t0 = time.perf_counter()
     oracle.transform_quant(w.x[:probe], w.P1, w.P2, w.cinv, w.alpha, w.n1, w.n2, nthreads=nth,
                            want_codes=False)
-    dt = time.perf_counter() - t0
-    per_tok = dt / probe
-    # tokens for about `seconds` of work: whole passes over the workload's rows
-    # when one pass is shorter than that, else its leading rows
-    sample = int(max(probe, seconds / max(per_tok, 1e-9)))
-    if max_tokens:
-        sample = min(sample, max_tokens)
-    done = 0
+    per_tok = (time.perf_counter() - t0) / probe
+    piece = int(max(probe, min(w.T, 1.0 / max(per_tok, 1e-9))))
+    done, row = 0, 0
     t0 = time.perf_counter()
-    while done < sample:
-        take = min(w.T, sample - done)
-        oracle.transform_quant(w.x[:take], w.P1, w.P2, w.cinv, w.alpha, w.n1, w.n2, nthreads=nth,
+    while True:
+        take = min(piece, w.T - row)
+        if max_tokens:
+            take = min(take, max_tokens - done)
+        oracle.transform_quant(w.x[row:row + take], w.P1, w.P2, w.cinv, w.alpha, w.n1, w.n2, nthreads=nth,
                                want_codes=False)
         done += take
-    el = time.perf_counter() - t0
-    return done / el, nth, done, el
+        row = (row + take) % w.T
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_tokens and done >= max_tokens):
+            return done / el, nth, done, el
 
 
 def run_reference(args):
