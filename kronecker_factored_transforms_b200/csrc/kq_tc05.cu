@@ -81,6 +81,7 @@ using namespace tc;
 using namespace tile;
 
 constexpr int kTcThreads = 768;  // 24 warps, at most 80 registers per thread
+constexpr int kSetupWarps = 15;  // warps 1, 5, 8-19, 21 build the factor operands
 constexpr int kXThreads = 256;   // x' split: warps 2-4, 6-7, 20, 22-23
 
 // Warp w runs on scheduler w % 4.  The x' split warps avoid scheduler 1, which
@@ -149,7 +150,13 @@ struct Cfg {
     static constexpr int SC = (SCALED && BUDGET >= 10 * XTILE) ? 4 : 2;  // lo-half tile stages (cinv)
     static constexpr int SX = imax(2, imin(8, (BUDGET - (SCALED ? SC * XTILE : 0)) / XTILE));  // raw x stages
     static constexpr int OFF_CONV = OFF_RAW + SX * XTILE;
-    static constexpr int NBAR = 2 * SX + 2 * SC + 3 * NB1 + 2 * NB2 + 1;
+    static constexpr int NBAR = 2 * SX + 2 * SC + 3 * NB1 + 2 * NB2 + 2;
+    // P1 and P2 arrive first, by bulk copies into the last NSCR x stages, which
+    // take x tiles only once the factor operands are built from them.
+    static constexpr int P1B = N1 * N1 * 2, P2B = N2 * N2 * 2;
+    static constexpr int OFF_SP2 = align_up(P1B, 1024);  // P2 within the scratch
+    static constexpr int NSCR = (OFF_SP2 + P2B + XTILE - 1) / XTILE;
+    static constexpr int OFF_SCR = OFF_RAW + (SX - NSCR) * XTILE;
     static constexpr int OFF_BAR = align_up(OFF_CONV + (SCALED ? SC * XTILE : 0), 16);
     static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem base, abort flag, the constant 1, 2 x 2 x 4 maxima
     static constexpr int SMEM = OFF_MISC + 80 + 1024;    // + slack for 1024-byte alignment
@@ -157,6 +164,8 @@ struct Cfg {
     static constexpr int FULL = 0, EMPTY = SX, CFULL = 2 * SX, CEMPTY = 2 * SX + SC;
     static constexpr int D1FULL = 2 * SX + 2 * SC, A2FULL = D1FULL + NB1, D1EMPTY = A2FULL + NB1;
     static constexpr int D2FULL = D1EMPTY + NB1, D2EMPTY = D2FULL + NB2, TEARDOWN = D2EMPTY + NB2;
+    static constexpr int FACT = TEARDOWN + 1;  // P1 and P2 landed in the scratch
+    static_assert(SX > NSCR, "at least one x stage besides the factor scratch");
     static_assert(N2 == 64 || N2 == 128, "stage 1 needs K = H * n2 = 128");
     static_assert(N1 % 16 == 0 && N1 >= 16 && N1 <= 128, "n1 must be a multiple of 16 in [16, 128]");
     static_assert(!SCALED || N1 <= 64, "x' split keeps cinv in registers: n1 <= 64");
@@ -240,6 +249,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(bar(C::D2EMPTY + b), 128);
         }
         mbar_init(bar(C::TEARDOWN), 2);  // one commit from each MMA issuer
+        mbar_init(bar(C::FACT), 1);
         *s_abort = 0;
         *reinterpret_cast<int *>(smem + C::OFF_MISC + 8) = 1;  // `one` of round_code
         fence_mbar_init();
@@ -253,17 +263,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_relinquish();
     }
 
-    // Barriers and the TMEM address are published.  The TMA producer and the x'
-    // split start at once; the other warps first build the factor operands, so
-    // that building them overlaps the first loads of x.
+    // Barriers and the TMEM address are published.  The TMA producer copies P1
+    // and P2 into the scratch stages first, then starts the stream of x tiles;
+    // the setup warps build the factor operands from the scratch while the x'
+    // split warps load cinv.
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     const int setup_idx = warp == 1 ? 0 : warp == 5 ? 1 : (warp >= 8 && warp < 20) ? warp - 6 : warp == 21 ? 14 : -1;
     if (setup_idx >= 0) {
-        constexpr int kSetupThreads = 15 * 32;
+        constexpr int kSetupThreads = kSetupWarps * 32;
         const int st = 32 * setup_idx + lane;
+        // P1 and P2 as the producer's first bulk copies put them in the scratch
+        // (on a timeout the abort flag is up and the operands do not matter)
+        wait_bounded(bar(C::FACT), 0u, s_abort, kSiteProducer, kWaitLimitNs, false);
+        const uint16_t *P1s = reinterpret_cast<const uint16_t *>(smem + C::OFF_SCR);
+        const uint16_t *P2s = reinterpret_cast<const uint16_t *>(smem + C::OFF_SCR + C::OFF_SP2);
         // B2[i][a] = P1[a][i] (rows i, K = a), 128B-swizzled K-major, zero beyond a = n1.
         {
             // A piece is one row i and eight consecutive a (zero past n1): eight
@@ -279,8 +295,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int a = a0 + 2 * e;
-                    const uint32_t lo = (c < PIECES && a < N1) ? P1[a * N1 + i] : 0u;
-                    const uint32_t hi = (c < PIECES && a + 1 < N1) ? P1[(a + 1) * N1 + i] : 0u;
+                    const uint32_t lo = (c < PIECES && a < N1) ? P1s[a * N1 + i] : 0u;
+                    const uint32_t hi = (c < PIECES && a + 1 < N1) ? P1s[(a + 1) * N1 + i] : 0u;
                     w[u][e] = lo | (hi << 16);
                 }
             }
@@ -302,7 +318,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int u = 0; u < PER; ++u) {
                 const int c = st + u * kSetupThreads;
-                if (c < PIECES) v[u] = *reinterpret_cast<const uint4 *>(P2 + 8 * c);
+                if (c < PIECES) v[u] = *reinterpret_cast<const uint4 *>(P2s + 8 * c);
             }
 #pragma unroll
             for (int u = 0; u < PER; ++u) {
@@ -332,21 +348,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int l = 32 * (warp & 3) + lane;
             const uint32_t taddr = tmem + (uint32_t(32 * (warp & 3)) << 16);
             const int kc0 = warp < 12 ? 0 : 2;
+            uint32_t w[2][16];  // every load first, then the two stores
 #pragma unroll
-            for (int kq = 0; kq < 2; ++kq) {
-                const int kc = kc0 + kq;
-                uint32_t w[16];
+            for (int kq = 0; kq < 2; ++kq)
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const int k = 32 * kc + 2 * e;
-                    w[e] = uint32_t(a1_value<N2>(P2, l, k)) | (uint32_t(a1_value<N2>(P2, l, k + 1)) << 16);
+                    const int k = 32 * (kc0 + kq) + 2 * e;
+                    w[kq][e] = uint32_t(a1_value<N2>(P2s, l, k)) | (uint32_t(a1_value<N2>(P2s, l, k + 1)) << 16);
                 }
-                tmem_st_32x32b_x16(taddr + 16 * kc, w);
-            }
+#pragma unroll
+            for (int kq = 0; kq < 2; ++kq) tmem_st_32x32b_x16(taddr + 16 * (kc0 + kq), w[kq]);
             tmem_wait_st();
         }
+        fence_proxy_async_smem();  // the scratch is read before TMA writes reuse it
         tc_fence_before();
-        named_barrier_sync(3, kSetupThreads);
+        named_barrier_sync(3, kSetupThreads + 32);  // with the TMA producer (warp 0)
         tc_fence_after();
     }
     // Buffer hand-offs from the tensor pipe are commits by the MMA warp: stage 1
@@ -356,11 +372,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 0) {
         // ---------------- TMA producer: one batch tile per slot ----------------
         // The whole warp runs the loop (converged); one elected lane issues.
+        // Its first copies are P1 and P2 (into the scratch stages), ahead of the
+        // stream of x tiles; the scratch stages take x tiles only after the
+        // setup warps have built the factor operands from them.
+        if (elect_one()) {
+            mbar_arrive_expect_tx(bar(C::FACT), uint32_t(C::P1B + C::P2B));
+            bulk_load(sbase + C::OFF_SCR, P1, uint32_t(C::P1B), bar(C::FACT));
+            bulk_load(sbase + C::OFF_SCR + C::OFF_SP2, P2, uint32_t(C::P2B), bar(C::FACT));
+        }
+        __syncwarp();
+        bool setup_seen = false;
         Ring rx;
         uint32_t issued = 0;
         int64_t g0 = int64_t(blockIdx.x) * C::GB;
         const int64_t gstep = int64_t(gridDim.x) * C::GB;
         for (int64_t j = 0; j < nb; ++j, g0 += gstep, rx.next(C::SX)) {
+            if (!setup_seen && j == C::SX - C::NSCR) {
+                named_barrier_sync(3, kSetupWarps * 32 + 32);
+                setup_seen = true;
+            }
             const bool ok = wait_bounded(bar(C::EMPTY + rx.idx), rx.phase ^ 1u, s_abort, kSiteProducer,
                                          kWaitLimitNs, false);
             if (!__all_sync(0xffffffffu, ok)) break;
@@ -382,7 +412,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             __syncwarp();
             ++issued;
         }
+        if (!setup_seen) named_barrier_sync(3, kSetupWarps * 32 + 32);  // fewer batches than free stages
         // Drain: every load issued has landed (the slots' last phases completed).
+        wait_bounded(bar(C::FACT), 0u, s_abort, kSiteDrain, kWaitLimitNs, true);
         Ring rd;
         for (uint32_t i = 0; i < issued; ++i, rd.next(C::SX))
             if (i + C::SX >= issued)
@@ -502,14 +534,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // arithmetic: hi = RN(x ch), lo = RN(x cl + RN(x ch - hi)).  Each step is one
             // fused rounding; hi + lo is x * cinv to about 2^-14 relative.
             uint32_t ch[UPT][4], cl[UPT][4];
+            float4 ca[UPT], cb[UPT];  // every load first
 #pragma unroll
             for (int u = 0; u < UPT; ++u) {
                 const int e = t + kXThreads * u;
                 const int c = e / (8 * N1), rem = e % (8 * N1), r = rem >> 3, up = rem & 7;
                 const int b0 = (N2 == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
-                const float4 ca = *reinterpret_cast<const float4 *>(cinv + r * N2 + b0);
-                const float4 cb = *reinterpret_cast<const float4 *>(cinv + r * N2 + b0 + 4);
-                const float cv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+                ca[u] = __ldg(reinterpret_cast<const float4 *>(cinv + r * N2 + b0));
+                cb[u] = __ldg(reinterpret_cast<const float4 *>(cinv + r * N2 + b0 + 4));
+            }
+#pragma unroll
+            for (int u = 0; u < UPT; ++u) {
+                const float cv[8] = {ca[u].x, ca[u].y, ca[u].z, ca[u].w, cb[u].x, cb[u].y, cb[u].z, cb[u].w};
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
                     const float c0 = cv[2 * p], c1 = cv[2 * p + 1];

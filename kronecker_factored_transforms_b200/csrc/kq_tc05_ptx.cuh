@@ -59,6 +59,13 @@ __device__ __forceinline__ void tma_store_2d(const void *tmap, int x, int y, uin
                  "r"(y), "r"(src)
                  : "memory");
 }
+// Untiled global -> shared copy of `bytes` (16-byte aligned, a multiple of 16),
+// completing as transaction bytes on mbarrier `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t sdst, const void *gsrc, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(sdst),
+                 "l"(gsrc), "r"(bytes), "r"(bar)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_store(void *gdst, uint32_t ssrc, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc),
                  "r"(bytes)
