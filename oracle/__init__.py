@@ -20,6 +20,11 @@ Parity status of each function (pins live in ``tests/test_oracle_pins.py``):
                     pinned: equals the Kronecker path with P1 = I (one row
                     per head), brute-force per-row quantisation, GQA head
                     counts.
+  e2m1_round, e4m3_round, nvfp4_quantize, headwise_transform_nvfp4
+                    pinned: the E2M1 and E4M3 value tables (count, extremes,
+                    subnormals), ties to even and saturation cases worked by
+                    hand, the quantiser's error bound and block-maximum
+                    invariants, a hand-computed row.
 """
 from __future__ import annotations
 
@@ -186,3 +191,126 @@ def headwise_transform_quant(x_bits, Ph_bits, alpha: float, heads: int, head_dim
     return dict(packed=r["packed"].reshape(T, heads * head_dim // 2), scale32=r["scale32"].reshape(T, heads),
                 scale64=r["scale64"].reshape(T, heads), codes=r["codes"].reshape(T, heads * head_dim),
                 dist=r["dist"].reshape(T, heads * head_dim))
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 (the 4-bit floating-point format with two levels of scale that the
+# FlatQuant page names as the direction it leaves open; the High-Rate
+# Quantized Matrix Multiplication page calls it a multi-scaled format with
+# group scaling).  Reading of the format: blocks of 16 consecutive values of a
+# row share one E4M3 scale; the elements are E2M1; each row has one fp32 scale.
+#
+# E2M1: sign, two exponent bits (bias 1), one mantissa bit; the magnitude code
+# m = 0 .. 7 encodes 0, 0.5, 1, 1.5, 2, 3, 4, 6.  E4M3: sign, four exponent
+# bits (bias 7), three mantissa bits, no infinities, magnitude code 0x7F is NaN:
+# the largest finite value is 1.75 * 2^8 = 448, subnormals are m / 8 * 2^-6.
+
+def e2m1_values() -> np.ndarray:
+    """Magnitudes of the E2M1 codes 0 .. 7, increasing."""
+    out = []
+    for m in range(8):
+        e, f = m >> 1, m & 1
+        out.append(0.5 * f if e == 0 else (1.0 + 0.5 * f) * 2.0 ** (e - 1))
+    return np.array(out)
+
+
+def e4m3_values() -> np.ndarray:
+    """Magnitudes of the finite E4M3 codes 0x00 .. 0x7E, increasing."""
+    out = []
+    for m in range(0x7F):
+        e, f = m >> 3, m & 7
+        out.append(f / 8.0 * 2.0 ** -6 if e == 0 else (1.0 + f / 8.0) * 2.0 ** (e - 7))
+    return np.array(out)
+
+
+def _round_to_table(a, table):
+    """Round non-negative a to the nearest entry of the increasing table (the
+    entry's index is the magnitude code); a tie goes to the even code; values
+    beyond the last entry saturate to it.  Returns (code, distance of a to the
+    nearest rounding boundary in units of the local step; inf when saturated
+    beyond the last entry)."""
+    a = np.asarray(a, dtype=np.float64)
+    top = table[-1]
+    sat = a >= top
+    ac = np.minimum(a, top)
+    hi = np.clip(np.searchsorted(table, ac, side="left"), 0, len(table) - 1)
+    lo = np.maximum(hi - 1, 0)
+    vh, vl = table[hi], table[lo]
+    dh, dl = vh - ac, ac - vl
+    pick_hi = (dh < dl) | ((dh == dl) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    step = np.where(hi > lo, vh - vl, 1.0)
+    mid = 0.5 * (vh + vl)
+    dist = np.where(hi > lo, np.abs(ac - mid) / step, np.inf)
+    dist = np.where(sat, np.inf, dist)
+    return code.astype(np.int64), dist
+
+
+def e2m1_round(a):
+    """Signed values -> 4-bit E2M1 codes (bit 3 the sign), round to nearest even,
+    saturating at +-6; also the distance to the nearest rounding boundary."""
+    a = np.asarray(a, dtype=np.float64)
+    m, dist = _round_to_table(np.abs(a), e2m1_values())
+    sign = (a < 0) & (m > 0)
+    return (m | (sign.astype(np.int64) << 3)).astype(np.uint8), dist
+
+
+def e4m3_round(a):
+    """Non-negative values -> E4M3 codes, round to nearest even, saturating at
+    448; also the distance to the nearest rounding boundary."""
+    m, dist = _round_to_table(np.asarray(a, dtype=np.float64), e4m3_values())
+    return m.astype(np.uint8), dist
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    c = np.asarray(codes, dtype=np.int64)
+    v = e2m1_values()[c & 7]
+    return np.where(c & 8, -v, v)
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    return e4m3_values()[np.asarray(codes, dtype=np.int64) & 0x7F]
+
+
+def nvfp4_quantize(y):
+    """NVFP4 of fp64 rows y [R, D] (D a multiple of 16), step by step:
+      1. row scale  s = max|y| / (6 * 448), rounded to fp32;
+      2. block scale  b = E4M3(max over the block of |y| / (6 s)), per 16 values;
+      3. element  q = E2M1(y / (decode(b) * s));
+      4. two codes per byte, element 2k in the low nibble.
+    A row (block) whose scale is zero gets zero block codes (element codes).
+    Returns dict(packed [R, D/2] uint8, codes [R, D] uint8, block [R, D/16] uint8,
+    scale32 [R] fp32, dist [R, D] (element rounding), bdist [R, D/16]
+    (block-scale rounding), value [R, D] (the decoded values))."""
+    y = np.asarray(y, dtype=np.float64)
+    R, D = y.shape
+    assert D % 16 == 0
+    s32 = (np.abs(y).max(axis=1) / (6.0 * 448.0)).astype(np.float32) if D else np.zeros(R, np.float32)
+    s = s32.astype(np.float64)
+    yb = y.reshape(R, D // 16, 16)
+    amax_b = np.abs(yb).max(axis=2)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        braw = np.where(s[:, None] > 0, amax_b / (6.0 * s[:, None]), 0.0)
+    bcode, bdist = e4m3_round(braw)
+    bdec = e4m3_decode(bcode)
+    den = bdec * s[:, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = np.where(den[:, :, None] > 0, yb / den[:, :, None], 0.0)
+    codes, dist = e2m1_round(r)
+    codes = codes.reshape(R, D)
+    dist = dist.reshape(R, D)
+    packed = (codes[:, 0::2] & 0xF) | ((codes[:, 1::2] & 0xF) << 4)
+    value = (e2m1_decode(codes).reshape(R, D // 16, 16) * den[:, :, None]).reshape(R, D)
+    return dict(packed=packed.astype(np.uint8), codes=codes, block=bcode, scale32=s32, dist=dist, bdist=bdist,
+                value=value)
+
+
+def headwise_transform_nvfp4(x_bits, Ph_bits, heads: int, head_dim: int):
+    """The per-head transform of ``headwise_transform_quant`` (rows x[t, h, :] times
+    the full factor Ph, fp64) followed by ``nvfp4_quantize`` of every (token,
+    head) row.  Returns the dict of ``nvfp4_quantize`` with rows (t, h) in order."""
+    x = np.asarray(x_bits, dtype=np.uint16).reshape(-1, heads * head_dim)
+    T = x.shape[0]
+    rows = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(T * heads, head_dim)
+    P = (np.asarray(Ph_bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return nvfp4_quantize(rows @ P.reshape(head_dim, head_dim))
