@@ -61,6 +61,8 @@ def parse():
                          "factors above 128 (--two-stage-config); headwise: the per-head key/value "
                          "transform + INT4 (8192 tokens x 32 heads x 128)")
     ap.add_argument("--two-stage-config", choices=["square65536", "ffn28672"], default="square65536")
+    ap.add_argument("--headwise-format", choices=["int4", "nvfp4"], default="int4",
+                    help="rows of the headwise workload: INT4 with one scale, or NVFP4 (E2M1, an E4M3 scale per 16)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0,
@@ -386,11 +388,17 @@ def run_headwise(args):
     Ph = Q.to(torch.bfloat16).contiguous()
     qs = [torch.empty((T, heads * D // 2), dtype=torch.uint8, device=dev) for _ in range(nset)]
     ss = [torch.empty((T, heads), dtype=torch.float32, device=dev) for _ in range(nset)]
+    fp4 = args.headwise_format == "nvfp4"
+    bs = [torch.empty((T, heads * D // 16), dtype=torch.uint8, device=dev) for _ in range(nset)] if fp4 else None
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
-        _lib.kq_headwise_transform_quant(xs[i % nset], Ph, 0.9, qs[i % nset], ss[i % nset], T, heads, D,
-                                         stream=stream.cuda_stream)
+        if fp4:
+            _lib.kq_headwise_transform_quant_nvfp4(xs[i % nset], Ph, qs[i % nset], bs[i % nset], ss[i % nset], T,
+                                                   heads, D, stream=stream.cuda_stream)
+        else:
+            _lib.kq_headwise_transform_quant(xs[i % nset], Ph, 0.9, qs[i % nset], ss[i % nset], T, heads, D,
+                                             stream=stream.cuda_stream)
 
     for i in range(max(3, args.warmup)):
         step(i)
@@ -407,13 +415,15 @@ def run_headwise(args):
         raise RuntimeError("a bounded wait timed out inside the kernel")
     ms = e0.elapsed_time(e1) / args.steps
     hbm_peak, _, kind = measured_peaks()
-    bytes_launch = R * (2 * D + D // 2 + 4)
+    bytes_launch = R * (2 * D + D // 2 + 4 + (D // 16 if fp4 else 0))
     achieved = bytes_launch / (ms / 1e3) / 1e9
-    line = {"metric": "rows/s and % HBM roofline of the per-head key/value transform + INT4", "value": R / (ms / 1e3),
+    fmt = "NVFP4" if fp4 else "INT4"
+    line = {"metric": "rows/s and %% HBM roofline of the per-head key/value transform + %s" % fmt, "value": R / (ms / 1e3),
             "unit": "rows/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "headwise: %d tokens x %d heads x head_dim %d, N(0,1) rows, orthogonal bf16 "
-                                   "factor, alpha 0.9" % (T, heads, D), "rows": R, "head_dim": D,
+                                   "factor, %s" % (T, heads, D, "NVFP4" if fp4 else "INT4, alpha 0.9"), "rows": R,
+                       "head_dim": D, "format": fmt,
                        "l2": "inputs rotate over %d buffer sets (%.0f MB > 2x L2)" % (nset, nset * set_bytes / 1e6)},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": None, "peak_source": "%s (MEASURED_PEAKS.json)" % kind,

@@ -154,6 +154,35 @@ kq_status kq_headwise_transform_quant(const uint16_t *x, const uint16_t *Ph, flo
                                       float *scale_out, int64_t T, int heads, int head_dim, kq_stream_t stream);
 
 /*
+ * kq_headwise_transform_quant_nvfp4 -- the per-head transform of
+ * kq_headwise_transform_quant with NVFP4 rows instead of INT4 (the 4-bit
+ * floating-point format with two levels of scale that the FlatQuant page
+ * leaves open; the High-Rate Quantized Matrix Multiplication page calls it a
+ * multi-scaled, group-scaled format).  For every row y = x[t, h, :] Ph of
+ * head_dim values:
+ *   row scale     s = max|y| / (6 * 448)                       (fp32)
+ *   block scale   b = E4M3(max over the block |y| / (6 s))     per 16 values,
+ *                 round to nearest even, saturating at 448
+ *   element       q = E2M1(y / (decode(b) * s)), round to nearest even,
+ *                 saturating at +-6; a value that rounds to zero is +0
+ * E2M1 codes: bit 3 the sign, magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6; two per
+ * byte, element 2k in the low nibble.  A row (block) with a zero scale has
+ * zero block (element) codes.
+ *
+ * x, Ph, T, heads, head_dim: as kq_headwise_transform_quant.
+ * q_out       [T, heads * head_dim / 2] device uint8, 16-byte aligned, written.
+ * block_scale_out [T, heads * head_dim / 16] device uint8 (E4M3 codes),
+ *             8-byte aligned, written.
+ * scale_out   [T, heads] device fp32, written.
+ * Returns KQ_ERR_SHAPE, KQ_ERR_UNSUPPORTED (head_dim), KQ_ERR_ARG (overlapping
+ * buffers), KQ_ERR_NULL, KQ_ERR_ALIGN, KQ_ERR_CUDA.  Asynchronous on
+ * `stream`; allocates nothing.
+ */
+kq_status kq_headwise_transform_quant_nvfp4(const uint16_t *x, const uint16_t *Ph, uint8_t *q_out,
+                                            uint8_t *block_scale_out, float *scale_out, int64_t T, int heads,
+                                            int head_dim, kq_stream_t stream);
+
+/*
  * kq_transform_quant_two_stage -- kq_transform_quant for factors up to 256
  * (FlatQuant page, "The fused kernel", Figure 8 (c): factors too large for one
  * on-chip pass; the transform runs as two stages with the intermediate in

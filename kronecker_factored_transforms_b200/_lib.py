@@ -45,9 +45,11 @@ def _load() -> ctypes.CDLL:
     lib.kq_headwise_transform_quant.argtypes = [P, P, F32, P, P, I64, I32, I32, P]
     lib.kq_transform_quant_two_stage.argtypes = [P, P, P, P, F32, P, P, P, ctypes.c_uint64, I64, I32, I32, P]
     lib.kq_transform_quant_two_stage_static.argtypes = [P, P, P, P, F32, P, P, I64, I32, I32, P]
+    lib.kq_headwise_transform_quant_nvfp4.argtypes = [P, P, P, P, P, I64, I32, I32, P]
     for f in (lib.kq_transform_quant, lib.kq_transform, lib.kq_dequant_inverse, lib.kq_device_error,
               lib.kq_selftest_bounded_wait, lib.kq_w4a4_gemm, lib.kq_headwise_transform_quant,
-              lib.kq_transform_quant_two_stage, lib.kq_transform_quant_two_stage_static):
+              lib.kq_transform_quant_two_stage, lib.kq_transform_quant_two_stage_static,
+              lib.kq_headwise_transform_quant_nvfp4):
         f.restype = ctypes.c_int
     lib.kq_two_stage_workspace_bytes.argtypes = [I64, I32, I32]
     lib.kq_two_stage_workspace_bytes.restype = ctypes.c_uint64
@@ -65,7 +67,7 @@ lib = _load()
 EXPORTED = ("kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_device_error",
             "kq_selftest_bounded_wait", "kq_status_string", "kq_kernel_name", "kq_version", "kq_w4a4_gemm",
             "kq_headwise_transform_quant", "kq_transform_quant_two_stage", "kq_two_stage_workspace_bytes",
-            "kq_transform_quant_two_stage_static")
+            "kq_transform_quant_two_stage_static", "kq_headwise_transform_quant_nvfp4")
 
 STATIC_WORKSPACE_BYTES = 64 * 1024 * 1024
 
@@ -124,6 +126,13 @@ def kq_transform_quant_two_stage_static(x, P1, P2, cinv, alpha: float, q_out, sc
     _check("kq_transform_quant_two_stage_static",
            lib.kq_transform_quant_two_stage_static(_ptr(x), _ptr(P1), _ptr(P2), _ptr(cinv), float(alpha), _ptr(q_out),
                                                    _ptr(scale_out), int(T), int(n1), int(n2), _stream(stream)))
+
+
+def kq_headwise_transform_quant_nvfp4(x, Ph, q_out, block_scale_out, scale_out, T: int, heads: int, head_dim: int,
+                                      stream=None) -> None:
+    _check("kq_headwise_transform_quant_nvfp4",
+           lib.kq_headwise_transform_quant_nvfp4(_ptr(x), _ptr(Ph), _ptr(q_out), _ptr(block_scale_out), _ptr(scale_out),
+                                                 int(T), int(heads), int(head_dim), _stream(stream)))
 
 
 def kq_w4a4_gemm(qx, sx, qw, sw, y, M: int, N: int, K: int, stream=None) -> None:

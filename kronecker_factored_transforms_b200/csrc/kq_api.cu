@@ -206,6 +206,33 @@ kq_status kq_headwise_transform_quant(const uint16_t *x, const uint16_t *Ph, flo
     return err == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;
 }
 
+kq_status kq_headwise_transform_quant_nvfp4(const uint16_t *x, const uint16_t *Ph, uint8_t *q_out,
+                                            uint8_t *block_scale_out, float *scale_out, int64_t T, int heads,
+                                            int head_dim, kq_stream_t stream) {
+    if (T < 0 || heads <= 0 || head_dim <= 0) return KQ_ERR_SHAPE;
+    if (head_dim != 64 && head_dim != 128) return KQ_ERR_UNSUPPORTED;
+    if (T > (int64_t(1) << 31) / heads) return KQ_ERR_SHAPE;  // rows are TMA coordinates
+    if (T == 0) return KQ_OK;
+    if (!x || !Ph || !q_out || !block_scale_out || !scale_out) return KQ_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(Ph, 16) || !aligned(q_out, 16) || !aligned(block_scale_out, 8) ||
+        !aligned(scale_out, 4))
+        return KQ_ERR_ALIGN;
+    const int64_t R = T * heads;
+    const Range in[2] = {range_of(x, uint64_t(R) * head_dim * 2), range_of(Ph, uint64_t(head_dim) * head_dim * 2)};
+    const Range out[3] = {range_of(q_out, uint64_t(R) * head_dim / 2), range_of(block_scale_out, uint64_t(R) * head_dim / 16),
+                          range_of(scale_out, uint64_t(R) * 4)};
+    for (const Range &o : out)
+        for (const Range &i : in)
+            if (overlap(o, i)) return KQ_ERR_ARG;
+    if (overlap(out[0], out[1]) || overlap(out[0], out[2]) || overlap(out[1], out[2])) return KQ_ERR_ARG;
+    DeviceInfo info;
+    kq_status st = device_info(info);
+    if (st != KQ_OK) return st;
+    cudaError_t err = kq::launch_rowwise_nvfp4(x, Ph, q_out, block_scale_out, scale_out, R, head_dim, info.num_sms,
+                                               info.device, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;
+}
+
 kq_status kq_transform_quant_two_stage(const uint16_t *x, const uint16_t *P1, const uint16_t *P2,
                                        const float *cinv, float alpha, uint8_t *q_out, float *scale_out,
                                        void *workspace, uint64_t workspace_bytes, int64_t T, int n1, int n2,

@@ -55,6 +55,11 @@ cudaError_t launch_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *
 // Per-head transform + INT4 per row: rows of head_dim (64 or 128) values.
 cudaError_t launch_rowwise(const uint16_t *x, const uint16_t *Ph, float alpha, uint8_t *q_out, float *scale_out,
                            int64_t R, int head_dim, int num_sms, int device, cudaStream_t stream);
+// The same transform with NVFP4 rows: E2M1 codes, an E4M3 scale per 16 values,
+// an fp32 scale per row.
+cudaError_t launch_rowwise_nvfp4(const uint16_t *x, const uint16_t *Ph, uint8_t *q_out, uint8_t *bscale_out,
+                                 float *scale_out, int64_t R, int head_dim, int num_sms, int device,
+                                 cudaStream_t stream);
 
 // Two-stage transform + INT4 for factors up to 256 through a workspace of
 // two_stage_workspace_bytes(T, n1, n2) bytes (Z^T hi then lo, bf16).

@@ -74,10 +74,46 @@ __device__ __forceinline__ uint32_t codes8(const uint32_t *v, float inv, int one
     return pack_s4x2(round_code_r(v[1], inv, one), round_code_r(v[0], inv, one), w);
 }
 
-template <int D>
+// ---- NVFP4: E2M1 elements, an E4M3 scale per 16 values, an fp32 scale per row --
+// Two fp32 values -> E4M3 codes (round to nearest even, saturating at 448): b in
+// the low byte, a in the high byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(a), "f"(b));
+    return d;
+}
+// The two E4M3 codes of e4m3x2 back to fp32 (exact).
+__device__ __forceinline__ void e4m3x2_decode(uint32_t c, float &lo, float &hi) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(uint16_t(c)));
+    lo = __half2float(__ushort_as_half(uint16_t(h2)));
+    hi = __half2float(__ushort_as_half(uint16_t(h2 >> 16)));
+}
+// Two fp32 values -> one byte of E2M1 codes (round to nearest even, saturating
+// at 6): b in the low nibble, a in the high nibble.
+__device__ __forceinline__ uint32_t e2m1x2(float a, float b) {
+    uint32_t d;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(d)
+        : "f"(a), "f"(b));
+    return d;
+}
+// Eight values times k -> a 32-bit word of E2M1 codes, value e in nibble e; a
+// value that rounds to zero is stored as +0 (the conversion keeps the sign).
+__device__ __forceinline__ uint32_t fp4x8(const uint32_t *v, float k) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+        w |= e2m1x2(__uint_as_float(v[2 * p + 1]) * k, __uint_as_float(v[2 * p]) * k) << (8 * p);
+    const uint32_t nz = (w | (w >> 1) | (w >> 2)) & 0x11111111u;  // nibbles with a nonzero magnitude
+    return w & (0x77777777u | (nz << 3));
+}
+
+template <int D, bool FP4>
 __global__ void __launch_bounds__(R_THREADS, 1)
     kq_rowwise_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint16_t *__restrict__ Ph, float alpha,
-                      uint8_t *__restrict__ q_out, float *__restrict__ scale_out, int64_t R, unsigned int *err) {
+                      uint8_t *__restrict__ q_out, float *__restrict__ scale_out, uint8_t *__restrict__ bscale_out,
+                      int64_t R, unsigned int *err) {
     using C = RCfg<D>;
     extern __shared__ __align__(1024) unsigned char r_raw[];
     const uint32_t raw_addr = smem_u32(r_raw);
@@ -216,10 +252,12 @@ __global__ void __launch_bounds__(R_THREADS, 1)
                 for (int e = 0; e < 32; e += 2)
                     m = fmax3(m, fabsf(__uint_as_float(v[e])), fabsf(__uint_as_float(v[e + 1])));
             }
-            const float sc = alpha * m * (1.0f / 7.0f);
+            // INT4: s = alpha max / 7.  NVFP4: the row scale s = max / (6 * 448).
+            const float sc = FP4 ? __fdiv_rn(m, 2688.0f) : alpha * m * (1.0f / 7.0f);
             const float inv = sc > 0.0f ? fminf(__fdividef(1.0f, sc), 3.0e38f) : 0.0f;
-            // pass 2: codes, 16 bytes per 32 values
+            // pass 2: codes, 16 bytes per 32 values (NVFP4: and one E4M3 scale per 16)
             uint8_t *qrow = q_out + row * (D / 2);
+            uint32_t bsc[D / 64 > 0 ? D / 64 : 1];  // the row's block-scale codes, four per word
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t v[32];
@@ -230,11 +268,41 @@ __global__ void __launch_bounds__(R_THREADS, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(C::DEMPTY + b));
                 }
-                const uint4 w = make_uint4(codes8(v, inv, one), codes8(v + 8, inv, one), codes8(v + 16, inv, one),
-                                           codes8(v + 24, inv, one));
+                uint4 w;
+                if constexpr (FP4) {
+                    // blocks 2c and 2c + 1: absmax, E4M3 scale code, element codes
+                    float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+                    for (int e = 0; e < 16; e += 2) {
+                        a0 = fmax3(a0, fabsf(__uint_as_float(v[e])), fabsf(__uint_as_float(v[e + 1])));
+                        a1 = fmax3(a1, fabsf(__uint_as_float(v[16 + e])), fabsf(__uint_as_float(v[17 + e])));
+                    }
+                    const uint32_t bc = e4m3x2(a1 * inv * (1.0f / 6.0f), a0 * inv * (1.0f / 6.0f));
+                    float d0, d1;
+                    e4m3x2_decode(bc, d0, d1);
+                    const float den0 = d0 * sc, den1 = d1 * sc;
+                    const float k0 = den0 > 0.0f ? __fdividef(1.0f, den0) : 0.0f;
+                    const float k1 = den1 > 0.0f ? __fdividef(1.0f, den1) : 0.0f;
+                    w = make_uint4(fp4x8(v, k0), fp4x8(v + 8, k0), fp4x8(v + 16, k1), fp4x8(v + 24, k1));
+                    if (c & 1)
+                        bsc[c >> 1] |= bc << 16;
+                    else
+                        bsc[c >> 1] = bc;
+                } else {
+                    w = make_uint4(codes8(v, inv, one), codes8(v + 8, inv, one), codes8(v + 16, inv, one),
+                                   codes8(v + 24, inv, one));
+                }
                 if (row < R) *reinterpret_cast<uint4 *>(qrow + 16 * c) = w;
             }
-            if (row < R) scale_out[row] = sc;
+            if (row < R) {
+                scale_out[row] = sc;
+                if constexpr (FP4) {
+                    if (D == 128)
+                        *reinterpret_cast<uint2 *>(bscale_out + row * (D / 16)) = make_uint2(bsc[0], bsc[1]);
+                    else
+                        *reinterpret_cast<uint32_t *>(bscale_out + row * (D / 16)) = bsc[0];
+                }
+            }
         }
     }
 
@@ -247,11 +315,11 @@ __global__ void __launch_bounds__(R_THREADS, 1)
     }
 }
 
-template <int D>
+template <int D, bool FP4>
 cudaError_t launch_rowwise_inst(const uint16_t *x, const uint16_t *Ph, float alpha, uint8_t *q_out, float *scale_out,
-                                int64_t R, int num_sms, int device, cudaStream_t stream) {
+                                uint8_t *bscale_out, int64_t R, int num_sms, int device, cudaStream_t stream) {
     using C = RCfg<D>;
-    auto kern = kq_rowwise_kernel<D>;
+    auto kern = kq_rowwise_kernel<D, FP4>;
     static std::once_flag once[64];
     static cudaError_t attr_err[64];
     if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
@@ -275,7 +343,7 @@ cudaError_t launch_rowwise_inst(const uint16_t *x, const uint16_t *Ph, float alp
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     const int64_t ntiles = (R + RT - 1) / RT;
     const int64_t grid = ntiles < num_sms ? ntiles : num_sms;
-    kern<<<unsigned(grid), R_THREADS, C::SMEM, stream>>>(tx, Ph, alpha, q_out, scale_out, R, err);
+    kern<<<unsigned(grid), R_THREADS, C::SMEM, stream>>>(tx, Ph, alpha, q_out, scale_out, bscale_out, R, err);
     return cudaGetLastError();
 }
 
@@ -284,8 +352,21 @@ cudaError_t launch_rowwise_inst(const uint16_t *x, const uint16_t *Ph, float alp
 cudaError_t launch_rowwise(const uint16_t *x, const uint16_t *Ph, float alpha, uint8_t *q_out, float *scale_out,
                            int64_t R, int head_dim, int num_sms, int device, cudaStream_t stream) {
     if (R >= (int64_t(1) << 31)) return cudaErrorInvalidValue;  // TMA row coordinate range
-    if (head_dim == 128) return launch_rowwise_inst<128>(x, Ph, alpha, q_out, scale_out, R, num_sms, device, stream);
-    if (head_dim == 64) return launch_rowwise_inst<64>(x, Ph, alpha, q_out, scale_out, R, num_sms, device, stream);
+    if (head_dim == 128)
+        return launch_rowwise_inst<128, false>(x, Ph, alpha, q_out, scale_out, nullptr, R, num_sms, device, stream);
+    if (head_dim == 64)
+        return launch_rowwise_inst<64, false>(x, Ph, alpha, q_out, scale_out, nullptr, R, num_sms, device, stream);
+    return cudaErrorNotSupported;
+}
+
+cudaError_t launch_rowwise_nvfp4(const uint16_t *x, const uint16_t *Ph, uint8_t *q_out, uint8_t *bscale_out,
+                                 float *scale_out, int64_t R, int head_dim, int num_sms, int device,
+                                 cudaStream_t stream) {
+    if (R >= (int64_t(1) << 31)) return cudaErrorInvalidValue;  // TMA row coordinate range
+    if (head_dim == 128)
+        return launch_rowwise_inst<128, true>(x, Ph, 1.0f, q_out, scale_out, bscale_out, R, num_sms, device, stream);
+    if (head_dim == 64)
+        return launch_rowwise_inst<64, true>(x, Ph, 1.0f, q_out, scale_out, bscale_out, R, num_sms, device, stream);
     return cudaErrorNotSupported;
 }
 

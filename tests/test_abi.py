@@ -30,7 +30,8 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for must in ("kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_status_string",
                  "kq_kernel_name", "kq_device_error", "kq_version", "kq_w4a4_gemm",
-                 "kq_headwise_transform_quant", "kq_transform_quant_two_stage", "kq_two_stage_workspace_bytes"):
+                 "kq_headwise_transform_quant", "kq_transform_quant_two_stage", "kq_two_stage_workspace_bytes",
+                 "kq_headwise_transform_quant_nvfp4"):
         assert must in names
 
 
@@ -148,6 +149,21 @@ def test_headwise_validation(kq):
     assert f(x, P, 0.9, q, q + 16, 4, 8, 128, None) == kq.KQ_ERR_ARG    # scales over codes
     assert f(None, None, 0.9, None, None, 0, 8, 128, None) == kq.KQ_OK  # empty: no-op
     assert f(x, P, 0.9, q, s_, 1 << 30, 8, 128, None) == kq.KQ_ERR_SHAPE
+
+
+def test_headwise_nvfp4_validation(kq):
+    f = kq.lib.kq_headwise_transform_quant_nvfp4
+    x, P, q, b, s_ = 0x100000, 0x200000, 0x300000, 0x380000, 0x400000
+    assert f(x, P, q, b, s_, -1, 8, 128, None) == kq.KQ_ERR_SHAPE
+    assert f(x, P, q, b, s_, 4, 8, 96, None) == kq.KQ_ERR_UNSUPPORTED
+    assert f(x, None, q, b, s_, 4, 8, 128, None) == kq.KQ_ERR_NULL
+    assert f(x, P, q, None, s_, 4, 8, 128, None) == kq.KQ_ERR_NULL
+    assert f(x, P, q, b + 4, s_, 4, 8, 128, None) == kq.KQ_ERR_ALIGN
+    assert f(x, P, q + 8, b, s_, 4, 8, 128, None) == kq.KQ_ERR_ALIGN
+    assert f(x, P, q, q + 64, s_, 4, 8, 128, None) == kq.KQ_ERR_ARG   # block scales over codes
+    assert f(x, P, x + 64, b, s_, 4, 8, 128, None) == kq.KQ_ERR_ARG   # codes over x
+    assert f(None, None, None, None, None, 0, 8, 128, None) == kq.KQ_OK
+    assert f(x, P, q, b, s_, 1 << 30, 8, 128, None) == kq.KQ_ERR_SHAPE
 
 
 def test_two_stage_validation(kq):
