@@ -48,7 +48,7 @@ typedef enum kq_status {
     KQ_OK = 0,
     KQ_ERR_NULL = -1,        /* a required pointer is NULL (with T > 0)             */
     KQ_ERR_SHAPE = -2,       /* T < 0, n1 <= 0, n2 <= 0, or T*n1*n2 overflows      */
-    KQ_ERR_UNSUPPORTED = -3, /* n1 or n2 not a multiple of 16 in [16, 128]         */
+    KQ_ERR_UNSUPPORTED = -3, /* a size or parameter the entry does not cover       */
     KQ_ERR_ALIGN = -4,       /* a pointer is not aligned as documented             */
     KQ_ERR_ARG = -5,         /* alpha not finite in (0, 1], or outputs overlap inputs */
     KQ_ERR_CUDA = -6,        /* a CUDA runtime call or a kernel launch failed      */

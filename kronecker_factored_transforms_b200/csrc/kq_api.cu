@@ -323,7 +323,9 @@ const char *kq_status_string(int status) {
     case KQ_OK: return "ok";
     case KQ_ERR_NULL: return "a required pointer is NULL";
     case KQ_ERR_SHAPE: return "bad shape (T < 0, n1 <= 0, n2 <= 0 or size overflow)";
-    case KQ_ERR_UNSUPPORTED: return "unsupported factor size (n1, n2 must be multiples of 16 in [16, 128])";
+    case KQ_ERR_UNSUPPORTED:
+        return "unsupported size or parameter for this entry (factors: multiples of 16 up to 128, or up to 256 for "
+               "the two-stage entries; head_dim 64 or 128; alpha of at least 2^-19 where the entry requires it)";
     case KQ_ERR_ALIGN: return "misaligned pointer";
     case KQ_ERR_ARG: return "bad argument (alpha outside (0, 1] or outputs overlap inputs)";
     case KQ_ERR_CUDA: return "CUDA runtime error";
