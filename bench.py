@@ -69,6 +69,9 @@ def parse():
                     help="CPU time the reference arm's warm-up + timed steps aim at")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling runs)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="token count of the transform workload instead of its own (profiling runs on a "
+                         "smaller case; the JSON line's config names the count used)")
     return ap.parse_args()
 
 
@@ -460,7 +463,7 @@ def main():
 
     from kronecker_factored_transforms_b200 import _lib
 
-    w = make_workload(WORKLOAD, shard=rank)
+    w = make_workload(WORKLOAD, T=args.tokens, shard=rank)
     T, n1, n2, n = w.T, w.n1, w.n2, w.n
     kernel = _lib.kq_kernel_name(n1, n2, w.cinv is not None)
 
@@ -585,7 +588,7 @@ def main():
     t_hbm = bytes_launch / (hbm_peak * 1e9)
     t_tc = flops_launch / (tf_peak * 1e12)
     roof = {"bound": "hbm" if t_hbm >= t_tc else "tensor", "achieved": achieved, "peak": hbm_peak,
-            "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": recorded_traffic(kernel),
+            "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": recorded_traffic(kernel) if args.tokens is None else None,
             "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
             else "fallback 6650 GB/s",
             "kernel": kernel, "bytes_per_launch": bytes_launch, "flops_per_launch": flops_launch,

@@ -598,25 +598,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             const uint32_t col0 = tmem + lane_off + C::R1(int(r1.idx));
             constexpr int NK = C::NS1 / 16;
-            constexpr int BATCH = NK < 2 ? NK : 2;
+            // Chunks of 16 columns, software-pipelined: chunk k + 1 is loaded while
+            // chunk k is converted and stored, so only the first load's latency is
+            // exposed.  (The wait ties the registers it makes valid, so no use of
+            // them is scheduled above it.)
+            uint32_t v[2][16];
+            tmem_ld_32x32b_x16(col0, v[0]);
+            tmem_wait_ld_tie(v[0]);
 #pragma unroll
-            for (int k0 = 0; k0 < NK; k0 += BATCH) {
-                uint32_t v[BATCH][16];
+            for (int k = 0; k < NK; ++k) {
+                if (k + 1 < NK) tmem_ld_32x32b_x16(col0 + 16 * (k + 1), v[(k + 1) & 1]);
+                // chunk of 16 columns -> 8 hi words then 8 lo words, in place
+                uint32_t o[16];
 #pragma unroll
-                for (int q = 0; q < BATCH; ++q)
-                    if (k0 + q < NK) tmem_ld_32x32b_x16(col0 + 16 * (k0 + q), v[q]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int q = 0; q < BATCH; ++q) {
-                    if (k0 + q < NK) {
-                        // chunk of 16 columns -> 8 hi words then 8 lo words, in place
-                        uint32_t o[16];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            split2(uint64_t(v[q][2 * e]) | (uint64_t(v[q][2 * e + 1]) << 32), o[e], o[8 + e]);
-                        tmem_st_32x32b_x16(col0 + 16 * (k0 + q), o);
-                    }
-                }
+                for (int e = 0; e < 8; ++e)
+                    split2(uint64_t(v[k & 1][2 * e]) | (uint64_t(v[k & 1][2 * e + 1]) << 32), o[e], o[8 + e]);
+                tmem_st_32x32b_x16(col0 + 16 * k, o);
+                if (k + 1 < NK) tmem_wait_ld_tie(v[(k + 1) & 1]);
             }
             tmem_wait_st();
             tc_fence_before();
