@@ -11,7 +11,7 @@ size 8192 factors as 64x128; LLaMA-2-7B hidden 4096) plus an FFN size of
 distributions (outlier channels, a pivot token, heavy tails, ReLU gating,
 per-channel scaling c) stand in for real LLM activations, which are not used.
 
-Conventions (one reading, fixed here and restated in the design doc):
+Conventions (one reading of the generator recipe, fixed here):
   * numpy ``default_rng(seed)`` (PCG64); draw order P1, P2, outlier channel
     set, c, then x (in chunks of ``CHUNK_ROWS`` rows).
   * shard r > 0 of a multi-GPU run draws its rows of x from
