@@ -29,6 +29,11 @@
  *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
  *     the legacy default stream).  Inputs are read-only; outputs must not
  *     overlap inputs (checked: KQ_ERR_ARG).
+ *   - The transform kernels are launched with programmatic stream
+ *     serialization: a launch may be scheduled while the previous kernel on
+ *     the stream (when that kernel allows it) is finishing, but it reads and
+ *     writes global memory only after that kernel has completed, so stream
+ *     order is kept for every buffer.
  *   - T == 0 is a no-op that returns KQ_OK without touching any pointer.
  *   - Arguments are checked before anything is launched; on error nothing
  *     runs and the status says why.  Faults inside a kernel surface at the

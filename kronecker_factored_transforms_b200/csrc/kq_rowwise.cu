@@ -120,6 +120,9 @@ __global__ void __launch_bounds__(R_THREADS, 1)
     const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
     unsigned char *smem = r_raw + (sbase - raw_addr);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // The next launch on the stream may be scheduled once every CTA has an SM
+    // (one CTA per SM, grid <= SMs); it waits for this grid before any global access.
+    griddep_launch_dependents();
     const int64_t ntiles = (R + RT - 1) / RT;
     auto bar = [&](int i) -> uint32_t { return sbase + uint32_t(C::OFF_BAR + 8 * i); };
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
@@ -143,6 +146,8 @@ __global__ void __launch_bounds__(R_THREADS, 1)
         tmem_alloc(sbase + C::OFF_MISC, 512);
         tmem_relinquish();
     }
+    // on-chip state only above; global reads and writes after the previous kernel
+    griddep_wait();
     // B = Ph^T in 128B-swizzled K-major chunks: row o (output column), K = k.
     // A unit is one row o and eight consecutive k: eight loads (consecutive
     // threads take consecutive o, so each load is coalesced), one 16-byte store
@@ -343,8 +348,8 @@ cudaError_t launch_rowwise_inst(const uint16_t *x, const uint16_t *Ph, float alp
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     const int64_t ntiles = (R + RT - 1) / RT;
     const int64_t grid = ntiles < num_sms ? ntiles : num_sms;
-    kern<<<unsigned(grid), R_THREADS, C::SMEM, stream>>>(tx, Ph, alpha, q_out, scale_out, bscale_out, R, err);
-    return cudaGetLastError();
+    return launch_overlapped(kern, unsigned(grid), R_THREADS, C::SMEM, stream, tx, Ph, alpha, q_out, scale_out,
+                             bscale_out, R, err);
 }
 
 }  // namespace

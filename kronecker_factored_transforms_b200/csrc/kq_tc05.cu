@@ -220,6 +220,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     unsigned char *smem = smem_raw + (sbase - raw_addr);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // The next launch on the stream may be scheduled once every CTA of this grid
+    // has got here, i.e. has an SM; with one CTA per SM its CTAs then take SMs
+    // as this grid's CTAs exit, and they wait for this grid's completion before
+    // touching global memory (griddep_wait below).
+    griddep_launch_dependents();
     // Work units: groups of H tokens; batches of GB groups, dealt round-robin to CTAs.
     const int64_t G = (T + C::H - 1) / C::H;
     const int64_t NBt = (G + C::GB - 1) / C::GB;
@@ -271,6 +276,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    // Everything above touched only on-chip state; every global read (x, P1, P2,
+    // cinv) and write (codes, scales) comes after the previous kernel on the
+    // stream has completed.
+    griddep_wait();
     const int setup_idx = warp == 1 ? 0 : warp == 5 ? 1 : (warp >= 8 && warp < 20) ? warp - 6 : warp == 21 ? 14 : -1;
     if (setup_idx >= 0) {
         constexpr int kSetupThreads = kSetupWarps * 32;
@@ -824,9 +833,11 @@ cudaError_t launch_inst(const LaunchArgs &a) {
     const int64_t G = (a.T + C::H - 1) / C::H;
     const int64_t NBt = (G + C::GB - 1) / C::GB;
     const int64_t grid = NBt < a.num_sms ? NBt : a.num_sms;
-    kern<<<unsigned(grid), kTcThreads, C::SMEM, a.stream>>>(tmap, tmap_q, a.P1, a.P2, a.cinv, a.alpha,
-                                                            a.scale_out, a.T);
-    return cudaGetLastError();
+    // Launched with programmatic stream serialization: when the previous kernel on
+    // the stream is another launch of this kernel, this grid's launch and set-up
+    // overlap that grid's last CTAs (see griddep_launch_dependents / griddep_wait).
+    return launch_overlapped(kern, unsigned(grid), kTcThreads, C::SMEM, a.stream, tmap, tmap_q, a.P1, a.P2, a.cinv,
+                             a.alpha, a.scale_out, a.T);
 }
 
 template <int N2, bool SCALED>

@@ -148,6 +148,9 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
     const uint32_t sbase = align1024(raw_addr);
     unsigned char *smem = s1_raw + (sbase - raw_addr);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // The next launch (stage 2) may be scheduled once every CTA has an SM (one
+    // CTA per SM, grid <= SMs); it waits for this grid before any global access.
+    griddep_launch_dependents();
     const int J = slices(n2), Jp = RT * J;
     const int rows = int(T * n1);                 // < 2^31 (checked by the entry)
     const int ntiles = (rows + R1 - 1) / R1;
@@ -187,6 +190,8 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + S1_OFF_MISC);
+    // on-chip state only above; global reads and writes after the previous kernel
+    griddep_wait();
 
     // P2 into shared memory first (row-major, the pipeline buffers are not in
     // use yet): 16-byte loads, eight per thread in flight.
@@ -489,6 +494,9 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
     unsigned char *smem = s2_raw + (sbase - raw_addr);
     const S2Layout L = s2_layout(n1, n2);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // The next launch may be scheduled once every CTA has an SM (one CTA per SM,
+    // grid <= SMs); it waits for this grid before any global access.
+    griddep_launch_dependents();
     const int n = n1 * n2, Jp = RT * L.J;
     auto bar = [&](int i) -> uint32_t { return sbase + uint32_t(L.off_bar + 8 * i); };
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L.off_misc + 4);
@@ -516,6 +524,9 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
         tmem_alloc(sbase + uint32_t(L.off_misc), 512);
         tmem_relinquish();
     }
+    // on-chip state only above; the workspace that stage 1 wrote, P1 and the
+    // outputs are touched only after the previous kernel (stage 1) has completed
+    griddep_wait();
     // B2 = P1^T in 128B-swizzled K-major chunks: row i, K = a; zero for a >= n1.
     // A unit is one row i and eight consecutive a: eight loads (consecutive
     // threads take consecutive i, so each load is coalesced), one 16-byte store
@@ -800,20 +811,14 @@ cudaError_t launch_two_stage(const LaunchArgs &a, void *workspace) {
     // stage 1: persistent CTAs over 64-row tiles
     const int64_t ntiles = (a.T * a.n1 + R1 - 1) / R1;
     const int64_t g1 = ntiles < a.num_sms ? ntiles : a.num_sms;
-    if (a.cinv)
-        kq_two_stage_s1_kernel<true><<<unsigned(g1), S1_THREADS, S1_SMEM, a.stream>>>(tx, tc, shi, slo, a.P2, a.T, a.n1,
-                                                                                      a.n2, err);
-    else
-        kq_two_stage_s1_kernel<false><<<unsigned(g1), S1_THREADS, S1_SMEM, a.stream>>>(tx, tc, shi, slo, a.P2, a.T,
-                                                                                       a.n1, a.n2, err);
-    e = cudaGetLastError();
+    e = launch_overlapped(a.cinv ? kq_two_stage_s1_kernel<true> : kq_two_stage_s1_kernel<false>, unsigned(g1),
+                          S1_THREADS, S1_SMEM, a.stream, tx, tc, shi, slo, a.P2, a.T, a.n1, a.n2, err);
     if (e != cudaSuccess) return e;
 
     // stage 2: one CTA per SM, tokens strided
     const int64_t g2 = a.T < a.num_sms ? a.T : a.num_sms;
-    kq_two_stage_s2_kernel<<<unsigned(g2), S2_THREADS, L.smem, a.stream>>>(lhi, llo, a.P1, a.alpha, a.q_out,
-                                                                           a.scale_out, a.T, a.n1, a.n2, err);
-    return cudaGetLastError();
+    return launch_overlapped(kq_two_stage_s2_kernel, unsigned(g2), S2_THREADS, size_t(L.smem), a.stream, lhi, llo,
+                             a.P1, a.alpha, a.q_out, a.scale_out, a.T, a.n1, a.n2, err);
 }
 
 }  // namespace kq
