@@ -40,6 +40,16 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Programmatic dependent launch.  launch_dependents: the next kernel on the
+// stream may be scheduled once every CTA of this grid has executed it (its CTAs
+// then start on SMs as this grid's CTAs exit).  wait: block until the previous
+// kernel's grid has completed and its memory operations are visible (returns at
+// once when the launch had no programmatic dependency).
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Launches `kern` with programmatic stream serialization: once every CTA of the
 // previous kernel on the stream has executed griddepcontrol.launch_dependents,
 // this grid may be scheduled, so its launch and on-chip set-up overlap that

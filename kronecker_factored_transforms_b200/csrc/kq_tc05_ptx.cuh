@@ -132,16 +132,6 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// Programmatic dependent launch.  launch_dependents: the next kernel on the
-// stream may be scheduled once every CTA of this grid has executed it (its CTAs
-// then start on SMs as this grid's CTAs exit).  wait: block until the previous
-// kernel's grid has completed and its memory operations are visible (returns at
-// once when the launch had no programmatic dependency).
-__device__ __forceinline__ void griddep_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // tcgen05.wait::ld that also names the 16 registers a load wrote, so that the
 // compiler schedules no read of them above the wait.
 __device__ __forceinline__ void tmem_wait_ld_tie(uint32_t (&r)[16]) {

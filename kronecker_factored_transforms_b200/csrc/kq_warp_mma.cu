@@ -107,6 +107,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *sRed = reinterpret_cast<float *>(smem + L.red);
     uint8_t *sOut = smem + L.out;
 
+    // The next launch on the stream may be scheduled once every CTA of this grid
+    // has started (the grid fits on the GPU at once); every global access below
+    // comes after the previous kernel on the stream has completed.
+    griddep_launch_dependents();
+    griddep_wait();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, q4 = lane & 3;
     const int slot = warp / G.wpt, jb = warp % G.wpt, j0 = 16 * jb;
@@ -345,9 +350,8 @@ cudaError_t launch_variant(const LaunchArgs &a) {
     const int64_t n_iter = (a.T + G.tpi - 1) / G.tpi;
     int64_t grid = int64_t(a.num_sms) * occ;
     if (grid > n_iter) grid = n_iter;
-    kern<<<static_cast<unsigned>(grid), kThreads, L.total, a.stream>>>(
-        a.x, a.P1, a.P2, a.cinv, a.alpha, a.q_out, a.scale_out, a.y_out, a.T, a.n1, a.n2);
-    return cudaGetLastError();
+    return launch_overlapped(kern, static_cast<unsigned>(grid), kThreads, L.total, a.stream, a.x, a.P1, a.P2, a.cinv,
+                             a.alpha, a.q_out, a.scale_out, a.y_out, a.T, a.n1, a.n2);
 }
 
 }  // namespace

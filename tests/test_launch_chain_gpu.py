@@ -29,13 +29,15 @@ def dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-def test_fused_chain_war_and_raw(kq):
-    w = make_workload("hidden8192", T=4096)          # 64 x 128 with cinv
-    T1, n1, n2, n = w.T, w.n1, w.n2, w.n
+@pytest.mark.parametrize("name,T1,T2", [("hidden8192", 4096, 8192),   # tcgen05 kernel, 64 x 128, cinv
+                                         ("tiny", 16384, 32768)])       # warp-MMA kernel, 16 x 16
+def test_transform_chain_war_and_raw(kq, name, T1, T2):
+    w = make_workload(name, T=T1)
+    n1, n2, n = w.n1, w.n2, w.n
     xA0 = dev(w.x.view(np.int16))
-    xB = dev(make_workload("hidden8192", T=8192, shard=1).x.view(np.int16))
-    P1, P2, cinv = dev(w.P1.view(np.int16)), dev(w.P2.view(np.int16)), dev(w.cinv)
-    T2 = 8192
+    xB = dev(make_workload(name, T=T2, shard=1).x.view(np.int16))
+    P1, P2 = dev(w.P1.view(np.int16)), dev(w.P2.view(np.int16))
+    cinv = dev(w.cinv) if w.cinv is not None else None
     T3 = T2 * (n // 2) // (2 * n)                     # call 2's codes read as bf16 rows of n
     q1, s1 = torch.empty(T1 * n // 2, dtype=torch.uint8, device="cuda"), torch.empty(T1, device="cuda")
     s2 = torch.empty(T2, device="cuda")
@@ -70,8 +72,8 @@ def test_fused_chain_war_and_raw(kq):
         call1(); call2(); call3()
         torch.cuda.synchronize()
         got = snap()
-        for name, g, r in zip(("q1", "s1", "q2", "s2", "q3", "s3"), got, ref):
-            assert torch.equal(g.view(torch.uint8), r.view(torch.uint8)), name
+        for label, g, r in zip(("q1", "s1", "q2", "s2", "q3", "s3"), got, ref):
+            assert torch.equal(g.view(torch.uint8), r.view(torch.uint8)), label
     assert kq.kq_device_error() == 0
 
 
@@ -115,6 +117,6 @@ def test_headwise_and_two_stage_chain(kq):
         for t in (qh1, sh1, q2, s2, qh3, sh3):
             t.fill_(0)
         got = chain(False)
-        for name, g, r in zip(("qh1", "sh1", "q2", "s2", "qh3", "sh3"), got, ref):
-            assert torch.equal(g.view(torch.uint8), r.view(torch.uint8)), name
+        for label, g, r in zip(("qh1", "sh1", "q2", "s2", "qh3", "sh3"), got, ref):
+            assert torch.equal(g.view(torch.uint8), r.view(torch.uint8)), label
     assert kq.kq_device_error() == 0
