@@ -235,7 +235,7 @@ class ClockSampler:
             pass
 
     def _loop(self):
-        while not self._stop.wait(0.02):
+        while not self._stop.wait(0.005):
             self.sample()
 
     def __enter__(self):
@@ -253,6 +253,9 @@ class ClockSampler:
         if not self.ok or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
         names = [k for k, v in self.REASONS.items() if self.reasons & v and k != "gpu_idle"]
+        other = self.reasons & ~sum(self.REASONS.values())
+        if other:
+            names.append("0x%x" % other)  # a reason bit this table does not name
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
                 "reasons": names, "samples": len(self.samples)}
 
