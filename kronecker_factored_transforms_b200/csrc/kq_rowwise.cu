@@ -120,9 +120,6 @@ __global__ void __launch_bounds__(R_THREADS, 1)
     const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
     unsigned char *smem = r_raw + (sbase - raw_addr);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // The next launch on the stream may be scheduled once every CTA has an SM
-    // (one CTA per SM, grid <= SMs); it waits for this grid before any global access.
-    griddep_launch_dependents();
     const int64_t ntiles = (R + RT - 1) / RT;
     auto bar = [&](int i) -> uint32_t { return sbase + uint32_t(C::OFF_BAR + 8 * i); };
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
@@ -173,6 +170,9 @@ __global__ void __launch_bounds__(R_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);
+    // The next launch may be scheduled once every CTA holds its SM and its TMEM;
+    // it touches global memory only after this grid completes.
+    griddep_launch_dependents();
 
     if (warp == 0) {
         // ---------------- TMA producer: x tiles [128 rows] x [D] ----------------

@@ -220,11 +220,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     unsigned char *smem = smem_raw + (sbase - raw_addr);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // The next launch on the stream may be scheduled once every CTA of this grid
-    // has got here, i.e. has an SM; with one CTA per SM its CTAs then take SMs
-    // as this grid's CTAs exit, and they wait for this grid's completion before
-    // touching global memory (griddep_wait below).
-    griddep_launch_dependents();
     // Work units: groups of H tokens; batches of GB groups, dealt round-robin to CTAs.
     const int64_t G = (T + C::H - 1) / C::H;
     const int64_t NBt = (G + C::GB - 1) / C::GB;
@@ -276,6 +271,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    // The next launch on the stream may be scheduled once every CTA of this grid
+    // has got here, i.e. holds its SM and its TMEM (so a CTA of that launch can
+    // never hold TMEM that this grid still waits for); its CTAs take SMs as this
+    // grid's CTAs exit and touch global memory only after this grid completes.
+    griddep_launch_dependents();
     // Everything above touched only on-chip state; every global read (x, P1, P2,
     // cinv) and write (codes, scales) comes after the previous kernel on the
     // stream has completed.

@@ -148,9 +148,6 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
     const uint32_t sbase = align1024(raw_addr);
     unsigned char *smem = s1_raw + (sbase - raw_addr);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // The next launch (stage 2) may be scheduled once every CTA has an SM (one
-    // CTA per SM, grid <= SMs); it waits for this grid before any global access.
-    griddep_launch_dependents();
     const int J = slices(n2), Jp = RT * J;
     const int rows = int(T * n1);                 // < 2^31 (checked by the entry)
     const int ntiles = (rows + R1 - 1) / R1;
@@ -190,6 +187,9 @@ __global__ void __launch_bounds__(S1_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + S1_OFF_MISC);
+    // The next launch (stage 2) may be scheduled once every CTA holds its SM and
+    // its TMEM; it touches global memory only after this grid completes.
+    griddep_launch_dependents();
     // on-chip state only above; global reads and writes after the previous kernel
     griddep_wait();
 
@@ -494,9 +494,6 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
     unsigned char *smem = s2_raw + (sbase - raw_addr);
     const S2Layout L = s2_layout(n1, n2);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // The next launch may be scheduled once every CTA has an SM (one CTA per SM,
-    // grid <= SMs); it waits for this grid before any global access.
-    griddep_launch_dependents();
     const int n = n1 * n2, Jp = RT * L.J;
     auto bar = [&](int i) -> uint32_t { return sbase + uint32_t(L.off_bar + 8 * i); };
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L.off_misc + 4);
@@ -565,6 +562,9 @@ __global__ void __launch_bounds__(S2_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + L.off_misc);
+    // The next launch may be scheduled once every CTA holds its SM and its TMEM;
+    // it touches global memory only after this grid completes.
+    griddep_launch_dependents();
 
     if (warp == 0) {
         // ---------------- TMA producer: Z^T hi/lo tiles [128 j] x [64 a] ----------------
