@@ -120,3 +120,39 @@ def test_headwise_and_two_stage_chain(kq):
         for label, g, r in zip(("qh1", "sh1", "q2", "s2", "qh3", "sh3"), got, ref):
             assert torch.equal(g.view(torch.uint8), r.view(torch.uint8)), label
     assert kq.kq_device_error() == 0
+
+
+def test_chain_in_a_cuda_graph(kq):
+    """The same kind of chain captured into a CUDA graph and replayed: every
+    output equals the eager, synchronised result."""
+    w = make_workload("llama7b_hidden", T=2048)      # 64 x 64, no cinv
+    n1, n2, n = w.n1, w.n2, w.n
+    x = dev(w.x.view(np.int16))
+    P1, P2 = dev(w.P1.view(np.int16)), dev(w.P2.view(np.int16))
+    T1 = w.T
+    q1, s1 = torch.empty(T1 * n // 2, dtype=torch.uint8, device="cuda"), torch.empty(T1, device="cuda")
+    T2 = T1 * (n // 2) // (2 * n)                     # call 1's codes read as bf16 rows of n
+    q2, s2 = torch.empty(T2 * n // 2, dtype=torch.uint8, device="cuda"), torch.empty(T2, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def chain():
+        kq.kq_transform_quant(x, P1, P2, None, w.alpha, q1, s1, T1, n1, n2, stream=stream)
+        kq.kq_transform_quant(q1, P1, P2, None, w.alpha, q2, s2, T2, n1, n2, stream=stream)
+
+    with torch.cuda.stream(stream):
+        chain()
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in (q1, s1, q2, s2)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        chain()
+    for _ in range(3):
+        for t in (q1, s1, q2, s2):
+            t.fill_(0)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        for label, a, b in zip(("q1", "s1", "q2", "s2"), (q1, s1, q2, s2), ref):
+            assert torch.equal(a.view(torch.uint8), b.view(torch.uint8)), label
+    del g
+    assert kq.kq_device_error() == 0
