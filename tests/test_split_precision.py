@@ -110,3 +110,29 @@ def test_e4m3_lo_candidate_uses_up_the_window(sample):
     shape = (S["T"], S["n1"], S["n2"])
     Z = hi.reshape(shape) @ S["P2"] + lo8.reshape(shape) @ P2b
     assert max_err(S, Z) > WINDOW / 2
+
+
+def test_two_stage_intermediate_needs_the_pair():
+    """The two-stage path keeps Z^T in its workspace as a hi + lo bf16 pair: on a
+    sample of the 256 x 256 workload a single bf16 Z leaves the window, the pair
+    does not."""
+    w = make_workload("square65536", rows=16)
+    T, n1, n2 = w.x.shape[0], w.n1, w.n2
+    widen = lambda bits: (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    x, P1, P2 = widen(w.x), widen(w.P1).reshape(n1, n1), widen(w.P2).reshape(n2, n2)
+    xp = (x * w.cinv.astype(np.float64)).reshape(T, n1, n2)
+    ref = oracle.transform_quant(w.x, w.P1, w.P2, w.cinv, w.alpha, n1, n2)
+    alpha = float(np.float32(w.alpha))
+    hi = bf16_rn(xp)
+    Z = hi @ P2 + bf16_rn(xp - hi) @ P2            # stage 1 with its own hi/lo operand
+
+    def outside(Zq):
+        Y = np.einsum("ai,taj->tij", P1, Zq).reshape(T, -1)
+        s = alpha * np.abs(Y).max(axis=1) / 7
+        q = np.clip(np.rint(Y / s[:, None]), -8, 7)
+        diff = q != ref["codes"]
+        return int((diff & ((np.abs(q - ref["codes"]) != 1) | (ref["dist"] >= WINDOW))).sum())
+
+    Zh = bf16_rn(Z)
+    assert outside(Zh) > 0
+    assert outside(Zh + bf16_rn(Z - Zh)) == 0
