@@ -200,3 +200,13 @@ def test_binding_raises_on_bad_status(kq):
     with pytest.raises(kq.KQError) as e:
         kq.kq_transform_quant(X, P1, P2, None, 0.9, Q, S, 4, 24, 16, stream=0)
     assert e.value.status == kq.KQ_ERR_UNSUPPORTED
+
+
+def test_build_covers_every_source_and_header():
+    """Every .cu file of csrc is compiled into libkq.so and every header counts
+    for the rebuild check, so no edit can leave a stale library behind."""
+    import os
+    from kronecker_factored_transforms_b200 import build as kb
+    files = set(os.listdir(kb.CSRC))
+    assert {f for f in files if f.endswith(".cu")} == set(kb.SOURCES)
+    assert {f for f in files if f.endswith((".cuh", ".h"))} == set(kb.HEADERS)
