@@ -67,6 +67,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0,
                     help="CPU time the reference arm's warm-up + timed steps aim at")
+    ap.add_argument("--sustained-ms", type=float, default=250.0,
+                    help="length of the sustained leg (back-to-back launches with their own clock record); 0 skips it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling runs)")
     ap.add_argument("--tokens", type=int, default=None,
@@ -137,6 +139,28 @@ def whole_job_tokens_per_s(world, tokens_per_rank, steps, ms):
 # ---------------------------------------------------------------------------
 # CPU oracle timing (baseline leg and the reference arm).
 
+def cpu_model():
+    """The host CPU's model name from /proc/cpuinfo (None where unavailable)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def cpu_fields():
+    """Host facts for a cpu_baseline record: the CPU model and the logical CPUs
+    the process may use (the oracle's thread count is reported as `cores`)."""
+    try:
+        avail = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        avail = os.cpu_count()
+    return {"cpu_model": cpu_model(), "hardware_concurrency": os.cpu_count(), "cpus_available": avail}
+
+
 def time_oracle(w, seconds, max_tokens=None):
     """The oracle on the host cores for about `seconds`: passes over the
     workload's rows, in pieces of about a second, until the time is reached
@@ -195,9 +219,9 @@ def run_reference(args):
             "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_dict(w, {"sample_tokens_per_step": sample}),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nth, "kind": "oracle",
-                             "sample": "first %d of %d tokens per step, fp64 C oracle, %d threads"
-                                       % (sample, w.T, nth)},
+            "cpu_baseline": dict({"value": value, "unit": UNIT, "cores": nth, "kind": "oracle",
+                                  "sample": "first %d of %d tokens per step, fp64 C oracle, %d threads"
+                                            % (sample, w.T, nth)}, **cpu_fields()),
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -514,6 +538,26 @@ def main():
     if world > 1:
         dist.barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1), dev, world)
+
+    # Sustained leg: the same launches back to back for about --sustained-ms, with
+    # a clock record of their own (a short timed region may see only boost
+    # clocks); reported beside `value`, which stays on the requested step count.
+    sustained = None
+    if args.sustained_ms > 0:
+        n_sus = max(args.steps, int(math.ceil(args.sustained_ms / max(ms / args.steps, 1e-3))))
+        sampler_sus = ClockSampler(dev.index if dev.index is not None else 0)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        with sampler_sus:
+            ev0.record(stream)
+            for i in range(n_sus):
+                step(i)
+            ev1.record(stream)
+            torch.cuda.synchronize(dev)
+        ms_sus = max_over_ranks(ev0.elapsed_time(ev1), dev, world)
+        sustained = {"launches": n_sus, "ms": ms_sus, "us_per_launch": 1e3 * ms_sus / n_sus,
+                     "clocks": sampler_sus.report()}
     if _lib.kq_device_error(stream) != 0:
         raise RuntimeError("a bounded wait timed out inside the kernel")
 
@@ -609,11 +653,17 @@ def main():
                    {"value": whole_job_tokens_per_s(world, T, args.e2e_steps, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps, "clocks": clocks}
+    if sustained is not None:
+        us = sustained["us_per_launch"]
+        sustained.update({"tokens_per_s": whole_job_tokens_per_s(world, T, sustained["launches"], sustained["ms"]),
+                          "achieved_gbs": bytes_launch / (us / 1e6) / 1e9,
+                          "frac": bytes_launch / (us / 1e6) / 1e9 / hbm_peak})
+        line["sustained"] = sustained
     if world == 1 and not args.no_cpu_baseline:
         v, cores, sample, el = time_oracle(w, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": "%d tokens (the workload's rows, repeated if needed) of %d per step, "
-                                          "fp64 C oracle, %.1f s" % (sample, T, el)}
+        line["cpu_baseline"] = dict({"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                     "sample": "%d tokens (the workload's rows, repeated if needed) of %d per step, "
+                                               "fp64 C oracle, %.1f s" % (sample, T, el)}, **cpu_fields())
     print(json.dumps(line), flush=True)
     return 0
 

@@ -235,8 +235,15 @@ kq_status kq_transform_quant_two_stage(const uint16_t *x, const uint16_t *P1, co
  * threads -- race on it and can return wrong codes; calls on one stream are
  * ordered and safe.  The first call on a device looks up the array's address
  * (cudaGetSymbolAddress, which can load the module) and must come before any
- * stream capture on that device.  Nothing is claimed about calling this entry
- * inside a captured graph.
+ * stream capture on that device; a lookup that fails is reported
+ * (KQ_ERR_CUDA) and tried again by the next call.  Nothing is claimed about
+ * calling this entry inside a captured graph.
+ *
+ * Device memory: under CUDA's default lazy module loading the 64 MiB are
+ * taken on a device when this entry is first called there, and kept until
+ * the process exits.  With CUDA_MODULE_LOADING=EAGER they are taken on every
+ * device the process creates a context on as soon as libkq is loaded, even if
+ * this entry is never called.
  */
 #define KQ_STATIC_WORKSPACE_BYTES (64ull * 1024ull * 1024ull)
 kq_status kq_transform_quant_two_stage_static(const uint16_t *x, const uint16_t *P1, const uint16_t *P2,

@@ -105,3 +105,47 @@ def test_headwise_nvfp4_is_rows_times_factor():
     ref = oracle.nvfp4_quantize(rows @ Pf)
     for k in ("packed", "block", "scale32"):
         np.testing.assert_array_equal(r[k], ref[k])
+
+
+def test_e2m1_boundary_distances():
+    """Distance to the nearest rounding boundary, in units of the local step
+    between the two neighbouring E2M1 magnitudes (the window the NVFP4 parity
+    test allows a one-step difference in).  Hand values: 2.5 is the midpoint of
+    2 and 3 (0); 2.75 is a quarter step above it (0.25); 5.5 lies between 4 and 6
+    (step 2, midpoint 5: 0.25); 0.3 between 0 and 0.5 (step 0.5, midpoint 0.25:
+    0.1); 1.0 sits on an entry, half a step from both boundaries (0.5); 3.375
+    between 3 and 4 (midpoint 3.5, step 1: 0.125); the sign does not matter;
+    6 and beyond saturate (inf: no boundary to be near)."""
+    a = np.array([2.5, 2.75, 5.5, 0.3, 1.0, 3.375, -2.75, 6.0, 9.0])
+    want = [0.0, 0.25, 0.25, 0.1, 0.5, 0.125, 0.25, np.inf, np.inf]
+    _, d = oracle.e2m1_round(a)
+    np.testing.assert_allclose(d, want, rtol=0, atol=1e-15)
+
+
+def test_e4m3_boundary_distances():
+    """The same for the E4M3 block scales: 1 + 1/16 is the midpoint of 1 and
+    1.125 (0); 1 + 3/32 a quarter step above it (0.25); in the binade [2, 4)
+    the step is 0.25, and 2.3125 lies between 2.25 and 2.5, a quarter step below
+    their midpoint 2.375 (0.25); 1.25 * 2^-9 between the subnormals 2^-9 and 2^-8 (step 2^-9, midpoint
+    1.5 * 2^-9: 0.25); 448 and beyond saturate (inf)."""
+    a = np.array([1 + 1 / 16, 1 + 3 / 32, 2.3125, 1.25 * 2.0 ** -9, 448.0, 500.0])
+    want = [0.0, 0.25, 0.25, 0.25, np.inf, np.inf]
+    _, d = oracle.e4m3_round(a)
+    np.testing.assert_allclose(d, want, rtol=0, atol=1e-15)
+
+
+def test_nvfp4_distances_follow_the_scaled_values():
+    """In nvfp4_quantize the element distance is taken on y / (block scale *
+    row scale) and the block distance on max|y| / (6 * row scale): one row,
+    built so that the row scale is 1 (max|y| = 6 * 448) and the second block's
+    raw scale 1 + 3/32 (block distance 0.25, as in the E4M3 table above), and an
+    element of the first block at 2.75 * 448 (element distance 0.25)."""
+    y = np.zeros((1, 32))
+    y[0, 0] = 6.0 * 448.0
+    y[0, 1] = 2.75 * 448.0
+    y[0, 16] = 6.0 * (1 + 3 / 32)
+    r = oracle.nvfp4_quantize(y)
+    assert r["scale32"][0] == 1.0
+    assert r["block"][0, 0] == 0x7E and r["bdist"][0, 0] == np.inf   # 448 saturates
+    assert r["bdist"][0, 1] == 0.25
+    assert r["dist"][0, 1] == 0.25

@@ -65,6 +65,12 @@ def test_golden_fixture(oracle_mod, path):
         assert r["scale64"][0] == pytest.approx(s, rel=1e-15)
         assert r["scale32"][0] == np.float32(s)
         assert oracle_mod.unpack_codes(r["packed"])[0].tolist() == case["codes"]
+        if "dist" in case:
+            # distances to the nearest rounding boundary, in units of y/s: exact binary
+            # fractions in these fixtures, so they must match exactly
+            assert r["dist"][0].tolist() == case["dist"]
+            q = oracle_mod.quantize(oracle_mod.transform(x, P1, P2, cinv, n1, n2), case["alpha"])
+            assert q["dist"][0].tolist() == case["dist"]
 
 
 def test_zero_token_gives_zero_scale_and_codes(oracle_mod):

@@ -153,7 +153,9 @@ def test_small_T(kq, T):
     assert_quant_parity(w.x, w.P1, w.P2, w.cinv, w.alpha, 64, 128, q, s)
 
 
-@pytest.mark.parametrize("alpha", [1.0, 0.5, 0.3, float(np.float32(1 / (1 + np.exp(-2.0))))])
+# 2^-19 is the smallest alpha the tcgen05 kernel takes (|y / s| <= 7 / alpha < 2^22 for
+# its rounding); 1e-7 goes to the warp-MMA kernel, where nearly every code saturates.
+@pytest.mark.parametrize("alpha", [1.0, 0.5, 0.3, float(np.float32(1 / (1 + np.exp(-2.0)))), 2.0 ** -19, 1e-7])
 def test_alpha_values(kq, alpha):
     w = make_workload("llama7b_hidden", rows=96)
     q, s = run_quant(kq, w.x, w.P1, w.P2, None, alpha, 96, 64, 64)

@@ -42,10 +42,14 @@ def test_static_workspace_rejects_oversize(kq):
 def test_static_workspace_matches_caller_workspace(kq):
     import torch
     dev16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
-    for call, (T, n1, n2, scaled) in enumerate([(9, 256, 256, True), (40, 112, 256, False)]):
+    # the last case fills the static array to its last byte: T = 256 at 256 x 256
+    cases = [(9, 256, 256, True), (40, 112, 256, False), (256, 256, 256, True)]
+    for call, (T, n1, n2, scaled) in enumerate(cases):
         x, P1, P2, cinv = _inputs(T, n1, n2, scaled, seed=31 + call)
         n = n1 * n2
         assert 4 * T * n <= kq.STATIC_WORKSPACE_BYTES
+        if call == 2:
+            assert kq.kq_two_stage_workspace_bytes(T, n1, n2) == kq.STATIC_WORKSPACE_BYTES
         xd, p1, p2 = dev16(x), dev16(P1), dev16(P2)
         cd = None if cinv is None else torch.from_numpy(cinv).cuda()
         need = kq.kq_two_stage_workspace_bytes(T, n1, n2)
