@@ -41,7 +41,8 @@ E2E_CHUNKS = 8  # chunks of a step in the end-to-end leg
 METRIC = "tokens/s and % roofline (HBM/tensor) for fused Kronecker transform+INT4 at n=8192"
 UNIT = "tokens/s"
 PROFILES = os.path.join(ROOT, "profiles")
-KERNEL_SOURCES = ["kronecker_factored_transforms_b200/csrc/kq_tc05.cu",
+KERNEL_SOURCES = ["kronecker_factored_transforms_b200/csrc/kq_fused.cu",
+                  "kronecker_factored_transforms_b200/csrc/kq_tc05.cu",
                   "kronecker_factored_transforms_b200/csrc/kq_tc05_ptx.cuh",
                   "kronecker_factored_transforms_b200/csrc/kq_warp_mma.cu",
                   "kronecker_factored_transforms_b200/csrc/kq_common.cuh",

@@ -9,8 +9,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libkq.so")
-SOURCES = ["kq_api.cu", "kq_warp_mma.cu", "kq_tc05.cu", "kq_inverse.cu", "kq_gemm.cu", "kq_rowwise.cu",
-           "kq_two_stage.cu", "kq_scratch.cu"]
+SOURCES = ["kq_api.cu", "kq_warp_mma.cu", "kq_tc05.cu", "kq_fused.cu", "kq_inverse.cu", "kq_gemm.cu",
+           "kq_rowwise.cu", "kq_two_stage.cu", "kq_scratch.cu"]
 HEADERS = ["kq_common.cuh", "kq_internal.h", "kq_tc05_ptx.cuh", "kq_tile.cuh", "kq_wait.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

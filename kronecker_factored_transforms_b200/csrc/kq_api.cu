@@ -87,10 +87,15 @@ kq_status run_transform(const uint16_t *x, const uint16_t *P1, const uint16_t *P
     a.device = info.device;
     a.stream = reinterpret_cast<cudaStream_t>(stream);
     // The tcgen05 kernel rounds with a 1.5 * 2^23 shift, exact while |y / s| = 7 / alpha < 2^22.
-    const bool fast = y_out == nullptr && alpha >= 0x1p-19f && kq::tc05_supports(n1, n2, cinv != nullptr);
-    cudaError_t err = fast
-                          ? kq::launch_tc05(a)
-                          : kq::launch_warp_mma(a);
+    const bool quant = y_out == nullptr && alpha >= 0x1p-19f;
+    const bool rows_ok = T * int64_t(n1) < (int64_t(1) << 31);  // TMA row coordinates are 32-bit
+    cudaError_t err;
+    if (quant && rows_ok && kq::fused_supports(n1, n2, cinv != nullptr))
+        err = kq::launch_fused(a);
+    else if (quant && kq::tc05_supports(n1, n2, cinv != nullptr))
+        err = kq::launch_tc05(a);
+    else
+        err = kq::launch_warp_mma(a);
     return err == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;
 }
 
@@ -336,6 +341,7 @@ const char *kq_status_string(int status) {
 
 const char *kq_kernel_name(int n1, int n2, int has_cinv) {
     if (!supported_factor(n1) || !supported_factor(n2)) return "unsupported";
+    if (kq::fused_supports(n1, n2, has_cinv != 0)) return "kq_fused_kernel";
     return kq::tc05_supports(n1, n2, has_cinv != 0) ? "kq_tc05_fused_kernel" : "kq_warp_mma_kernel";
 }
 

@@ -31,6 +31,10 @@ cudaError_t launch_warp_mma(const LaunchArgs &a);
 bool tc05_supports(int n1, int n2, bool scaled);
 cudaError_t launch_tc05(const LaunchArgs &a);
 
+// Group-pipelined tcgen05/TMEM kernel (n1 = 64, n2 in {64, 128}; alpha >= 2^-19).
+bool fused_supports(int n1, int n2, bool scaled);
+cudaError_t launch_fused(const LaunchArgs &a);
+
 // Diagnostic: a kernel whose bounded wait on a never-signalled barrier gives up.
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
 
