@@ -493,7 +493,7 @@ def main():
 
     w = make_workload(WORKLOAD, T=args.tokens, shard=rank)
     T, n1, n2, n = w.T, w.n1, w.n2, w.n
-    kernel = _lib.kq_kernel_name(n1, n2, w.cinv is not None)
+    kernel = _lib.kq_kernel_for(T, n1, n2, w.cinv is not None, w.alpha)
 
     # Rotating device buffer sets: total > 2x L2 so x comes from HBM every step.
     props = torch.cuda.get_device_properties(dev)

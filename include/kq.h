@@ -278,10 +278,19 @@ kq_status kq_selftest_bounded_wait(int64_t limit_us, kq_stream_t stream);
 const char *kq_status_string(int status);
 
 /*
- * Name of the kernel kq_transform_quant launches for this shape (static
- * storage), or "unsupported".  Host-only; touches no device state.
+ * Name of the kernel kq_transform_quant launches for this shape on long inputs
+ * (static storage), or "unsupported".  Host-only; touches no device state.
  */
 const char *kq_kernel_name(int n1, int n2, int has_cinv);
+
+/*
+ * Name of the kernel kq_transform_quant launches for this call size (T tokens)
+ * and clip ratio on the current device (static storage), or "unsupported".
+ * Short launches of n1 = 64 (at most 24 groups of 128/n2 tokens per SM) run
+ * kq_fused_kernel, the group-pipelined kernel; longer ones the kernel that
+ * kq_kernel_name names.  Reads the device's SM count; launches nothing.
+ */
+const char *kq_kernel_for(int64_t T, int n1, int n2, int has_cinv, float alpha);
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int kq_version(void);

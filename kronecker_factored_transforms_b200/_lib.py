@@ -57,6 +57,8 @@ def _load() -> ctypes.CDLL:
     lib.kq_status_string.restype = ctypes.c_char_p
     lib.kq_kernel_name.argtypes = [I32, I32, I32]
     lib.kq_kernel_name.restype = ctypes.c_char_p
+    lib.kq_kernel_for.argtypes = [I64, I32, I32, I32, ctypes.c_float]
+    lib.kq_kernel_for.restype = ctypes.c_char_p
     lib.kq_version.argtypes = []
     lib.kq_version.restype = ctypes.c_int
     return lib
@@ -65,7 +67,7 @@ def _load() -> ctypes.CDLL:
 lib = _load()
 
 EXPORTED = ("kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_device_error",
-            "kq_selftest_bounded_wait", "kq_status_string", "kq_kernel_name", "kq_version", "kq_w4a4_gemm",
+            "kq_selftest_bounded_wait", "kq_status_string", "kq_kernel_name", "kq_kernel_for", "kq_version", "kq_w4a4_gemm",
             "kq_headwise_transform_quant", "kq_transform_quant_two_stage", "kq_two_stage_workspace_bytes",
             "kq_transform_quant_two_stage_static", "kq_headwise_transform_quant_nvfp4")
 
@@ -169,6 +171,10 @@ def kq_status_string(status: int) -> str:
 
 def kq_kernel_name(n1: int, n2: int, has_cinv: bool) -> str:
     return lib.kq_kernel_name(int(n1), int(n2), int(bool(has_cinv))).decode()
+
+
+def kq_kernel_for(T: int, n1: int, n2: int, has_cinv: bool, alpha: float = 0.9) -> str:
+    return lib.kq_kernel_for(int(T), int(n1), int(n2), int(bool(has_cinv)), float(alpha)).decode()
 
 
 def kq_version() -> int:

@@ -179,16 +179,18 @@ struct Cfg {
 };
 
 // v = hi + lo with hi = v truncated to bf16 (its top 16 bits, a byte permute)
-// and lo = v - hi (exact in fp32) rounded to bf16 (one conversion per pair):
-// about 16 significant bits in all.  Takes two fp32 values as one 64-bit
-// pair; returns the two hi values packed (first in the low half) and the two
-// lo ones.
-__device__ __forceinline__ void split2(uint64_t v, uint32_t &hi, uint32_t &lo) {
-    const uint32_t v0 = uint32_t(v), v1 = uint32_t(v >> 32);
-    const uint64_t t = uint64_t(v0 & 0xFFFF0000u) | (uint64_t(v1 & 0xFFFF0000u) << 32);
-    const uint64_t l = f32x2_sub(v, t);
+// and lo = v - hi (exact in fp32) rounded to bf16: about 16 significant bits in
+// all.  Returns the two hi values packed (first in the low half) and the two
+// NEGATED lo values: hi - v is one mixed bf16/fp32 subtraction per value, and
+// stage 2 multiplies the lo half by -P1^T (the MMA's negate-B bit).
+__device__ __forceinline__ void split_pair_neg(uint32_t v0, uint32_t v1, uint32_t &hi, uint32_t &nlo) {
     hi = __byte_perm(v0, v1, 0x7632);
-    lo = pack_bf16x2(__uint_as_float(uint32_t(l)), __uint_as_float(uint32_t(l >> 32)));
+    float n0, n1;
+    asm("{\n\t.reg .b16 h0, h1;\n\tmov.b32 {h0, h1}, %2;\n\t"
+        "sub.rn.f32.bf16 %0, h0, %3;\n\tsub.rn.f32.bf16 %1, h1, %4;\n\t}"
+        : "=f"(n0), "=f"(n1)
+        : "r"(hi), "f"(__uint_as_float(v0)), "f"(__uint_as_float(v1)));
+    nlo = pack_bf16x2(n0, n1);
 }
 
 // round_half_even(y * inv) as an int, valid for |y * inv| < 2^22 (alpha >= 2^-19):
@@ -198,11 +200,14 @@ __device__ __forceinline__ void split2(uint64_t v, uint32_t &hi, uint32_t &lo) {
 // work instead of on the logic pipe.  (A packed fp32x2 form needs register
 // pairs the TMEM loads do not provide, and costs more instructions.)
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;  // 1.5 * 2^23
-__device__ __forceinline__ int round_code(uint32_t ybits, float inv, int one) {
-    const uint32_t b = __float_as_uint(fmaf(__uint_as_float(ybits), inv, 12582912.0f));
-    int k;
-    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k) : "r"(b), "r"(one), "r"(-int(kRoundMagicBits)));
-    return k;
+// Two values at once: one packed fp32x2 multiply-add, then the two offsets removed.
+__device__ __forceinline__ void round_code2(uint32_t y0, uint32_t y1, uint64_t inv2, int one, int &k0, int &k1) {
+    const uint64_t y = uint64_t(y0) | (uint64_t(y1) << 32);
+    const uint64_t magic = (uint64_t(kRoundMagicBits) << 32) | kRoundMagicBits;
+    uint64_t b;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(b) : "l"(y), "l"(inv2), "l"(magic));
+    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k0) : "r"(uint32_t(b)), "r"(one), "r"(-int(kRoundMagicBits)));
+    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k1) : "r"(uint32_t(b >> 32)), "r"(one), "r"(-int(kRoundMagicBits)));
 }
 
 
@@ -437,6 +442,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // covers the MMAs its own thread issued.
         constexpr uint32_t idesc1 = idesc_bf16_f32(128, C::NS1);
         constexpr uint32_t idesc2 = idesc_bf16_f32(128, N1);
+        // The A2 lo half holds -lo (split_pair_neg): stage 2 negates B on the lo pass.
+        constexpr uint32_t idesc2n = idesc2 | (1u << 14);
         const uint32_t b2l = sdesc_sw128_lo(sbase + C::OFF_B2);
         const uint64_t a1d = sdesc_kmajor_sw128(sbase + C::OFF_A1);
         // descriptor start addresses are in 16-byte units in the low bits
@@ -468,17 +475,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
                             const uint32_t b = (pass ? bl_lo : bl_hi) + koff1(kk);
+                            const uint32_t id1 = idesc1;
                             if (C::A1_TMEM) {
                                 if ((pass | kk) != 0)
-                                    mma_ts_split<1>(d1, tmem + 8 * kk, b, kSdescSw128Hi, idesc1);
+                                    mma_ts_split<1>(d1, tmem + 8 * kk, b, kSdescSw128Hi, id1);
                                 else
-                                    mma_ts_split<0>(d1, tmem + 8 * kk, b, kSdescSw128Hi, idesc1);
+                                    mma_ts_split<0>(d1, tmem + 8 * kk, b, kSdescSw128Hi, id1);
                             } else {
                                 const uint64_t a = a1d + uint64_t(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
                                 if ((pass | kk) != 0)
-                                    mma_ss_split<1>(d1, a, b, kSdescSw128Hi, idesc1);
+                                    mma_ss_split<1>(d1, a, b, kSdescSw128Hi, id1);
                                 else
-                                    mma_ss_split<0>(d1, a, b, kSdescSw128Hi, idesc1);
+                                    mma_ss_split<0>(d1, a, b, kSdescSw128Hi, id1);
                             }
                         }
                     }
@@ -511,7 +519,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             for (int kk = 0; kk < N1 / 16; ++kk) {
                                 if ((pass | kk) != 0)
                                     mma_ts_split<1>(d2, a2 + 16 * kk + 8 * pass, b2l + koff2(kk), kSdescSw128Hi,
-                                                    idesc2);
+                                                    pass ? idesc2n : idesc2);
                                 else
                                     mma_ts_split<0>(d2, a2 + 16 * kk + 8 * pass, b2l + koff2(kk), kSdescSw128Hi,
                                                     idesc2);
@@ -617,11 +625,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int k = 0; k < NK; ++k) {
                 if (k + 1 < NK) tmem_ld_32x32b_x16(col0 + 16 * (k + 1), v[(k + 1) & 1]);
-                // chunk of 16 columns -> 8 hi words then 8 lo words, in place
+                // chunk of 16 columns -> 8 hi words then 8 -lo words, in place
                 uint32_t o[16];
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    split2(uint64_t(v[k & 1][2 * e]) | (uint64_t(v[k & 1][2 * e + 1]) << 32), o[e], o[8 + e]);
+                    split_pair_neg(v[k & 1][2 * e], v[k & 1][2 * e + 1], o[e], o[8 + e]);
                 tmem_st_32x32b_x16(col0 + 16 * k, o);
                 if (k + 1 < NK) tmem_wait_ld_tie(v[(k + 1) & 1]);
             }
@@ -719,6 +727,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // exact quotients by a few ulps, far inside the rounding-boundary window
             const float s = alpha * m * (1.0f / 7.0f);
             const float inv = s > 0.0f ? fminf(__fdividef(1.0f, s), 3.0e38f) : 0.0f;
+            const uint64_t inv2 = (uint64_t(__float_as_uint(inv)) << 32) | __float_as_uint(inv);
             unsigned char *stg = smem + C::OFF_STG + (2 * ew + buf) * C::STG;
             // this thread's two bytes of every row: columns 4 g8 .. 4 g8 + 3 of the warp's 32.
             // It writes rows row0 + 16 c + 8 rep + 2 qq + d, whose swizzle term of
@@ -750,14 +759,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int rep = 0; rep < 2 * CB; ++rep) {
                     // rows i0 + d, i0 = 16 c0 + 8 rep + 2 qq: registers 4 rep + d hold the even
                     // column, 4 rep + 2 + d the odd one, of half 0 (ra) and half 1 (rb)
+                    int ka[4], kb[4];
+                    round_code2(ra[4 * rep], ra[4 * rep + 1], inv2, one, ka[0], ka[1]);
+                    round_code2(ra[4 * rep + 2], ra[4 * rep + 3], inv2, one, ka[2], ka[3]);
+                    round_code2(rb[4 * rep], rb[4 * rep + 1], inv2, one, kb[0], kb[1]);
+                    round_code2(rb[4 * rep + 2], rb[4 * rep + 3], inv2, one, kb[2], kb[3]);
 #pragma unroll
                     for (int d = 0; d < 2; ++d) {
                         // row i0 + d: columns 4 g8 + (0, 1) from half 0, + (2, 3) from half 1;
                         // byte = even column in the low nibble, odd in the high one
-                        const uint32_t wb = pack_s4x2(round_code(rb[4 * rep + 2 + d], inv, one),
-                                                      round_code(rb[4 * rep + d], inv, one), 0u);
-                        const uint32_t w = pack_s4x2(round_code(ra[4 * rep + 2 + d], inv, one),
-                                                     round_code(ra[4 * rep + d], inv, one), wb);
+                        const uint32_t wb = pack_s4x2(kb[2 + d], kb[d], 0u);
+                        const uint32_t w = pack_s4x2(ka[2 + d], ka[d], wb);
                         *reinterpret_cast<uint16_t *>(tbase + (16 * c0 + 8 * rep + d) * C::RB) = uint16_t(w);
                     }
                 }

@@ -244,8 +244,15 @@ def test_dequant_inverse_matches_oracle_and_round_trips(kq):
 # Kernel selection and the bounded-wait failure path.
 
 def test_fast_kernel_is_selected_for_the_configs(kq):
+    # long launches: the batch-pipelined kernel; short ones of n1 = 64: the group-pipelined one
     for n1, n2, scaled in [(64, 64, False), (64, 128, True), (112, 128, False)]:
         assert kq.kq_kernel_name(n1, n2, scaled) == "kq_tc05_fused_kernel"
+    assert kq.kq_kernel_for(8192, 64, 128, True, 0.85) == "kq_tc05_fused_kernel"   # hidden8192
+    assert kq.kq_kernel_for(65536, 64, 64, False, 0.9) == "kq_tc05_fused_kernel"   # sweep4096, largest T
+    assert kq.kq_kernel_for(2048, 64, 64, False, 0.88) == "kq_fused_kernel"        # llama7b_hidden
+    assert kq.kq_kernel_for(1, 64, 128, True, 0.85) == "kq_fused_kernel"
+    assert kq.kq_kernel_for(4096, 112, 128, False, 0.9) == "kq_tc05_fused_kernel"  # mlp14336
+    assert kq.kq_kernel_for(64, 64, 64, False, 1e-7) == "kq_warp_mma_kernel"
     assert kq.kq_kernel_name(16, 16, False) == "kq_warp_mma_kernel"
 
 
