@@ -152,11 +152,16 @@ struct Cfg {
     static constexpr int OFF_CONV = OFF_RAW + SX * XTILE;
     static constexpr int NBAR = 2 * SX + 2 * SC + 3 * NB1 + 2 * NB2 + 2;
     // P1 and P2 arrive first, by bulk copies into the last NSCR x stages, which
-    // take x tiles only once the factor operands are built from them.
+    // take x tiles only once the factor operands are built from them.  With cinv
+    // and n1 >= 112 only two x stages fit; the scratch then takes the lo-half
+    // stages that follow them (SCR_CONV), which the split warps fill only after
+    // the factor operands are built.
     static constexpr int P1B = N1 * N1 * 2, P2B = N2 * N2 * 2;
     static constexpr int OFF_SP2 = align_up(P1B, 1024);  // P2 within the scratch
     static constexpr int NSCR = (OFF_SP2 + P2B + XTILE - 1) / XTILE;
-    static constexpr int OFF_SCR = OFF_RAW + (SX - NSCR) * XTILE;
+    static constexpr bool SCR_CONV = SCALED && SX <= NSCR;
+    static constexpr int NSCR_RAW = SCR_CONV ? imax(0, NSCR - SC) : NSCR;  // x stages in the scratch
+    static constexpr int OFF_SCR = OFF_RAW + (SX + (SCR_CONV ? SC : 0) - NSCR) * XTILE;
     static constexpr int OFF_BAR = align_up(OFF_CONV + (SCALED ? SC * XTILE : 0), 16);
     static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem base, abort flag, the constant 1, 2 x 2 x 4 maxima
     static constexpr int SMEM = OFF_MISC + 80 + 1024;    // + slack for 1024-byte alignment
@@ -165,10 +170,9 @@ struct Cfg {
     static constexpr int D1FULL = 2 * SX + 2 * SC, A2FULL = D1FULL + NB1, D1EMPTY = A2FULL + NB1;
     static constexpr int D2FULL = D1EMPTY + NB1, D2EMPTY = D2FULL + NB2, TEARDOWN = D2EMPTY + NB2;
     static constexpr int FACT = TEARDOWN + 1;  // P1 and P2 landed in the scratch
-    static_assert(SX > NSCR, "at least one x stage besides the factor scratch");
+    static_assert(SX > NSCR_RAW && NSCR - NSCR_RAW <= (SCALED ? SC : 0) , "at least one x stage besides the factor scratch");
     static_assert(N2 == 64 || N2 == 128, "stage 1 needs K = H * n2 = 128");
     static_assert(N1 % 16 == 0 && N1 >= 16 && N1 <= 128, "n1 must be a multiple of 16 in [16, 128]");
-    static_assert(!SCALED || N1 <= 64, "x' split keeps cinv in registers: n1 <= 64");
     static_assert(NS1 % 16 == 0 && NS1 <= 128, "stage-1 MMA width");
     static_assert(NB1 >= 2, "stage-1 regions");
     static_assert(TMEM_USED <= 512, "TMEM budget");
@@ -177,6 +181,13 @@ struct Cfg {
     __host__ __device__ static constexpr uint32_t R1(int b) { return uint32_t(A1COLS + b * R1W); }
     __host__ __device__ static constexpr uint32_t R2(int b) { return uint32_t(A1COLS + NB1 * R1W + b * N1P); }
 };
+
+// Threads of the named barrier that ends the setup: the setup warps, the TMA
+// producer and, when the factor scratch overlaps the lo-half stages, the split warps.
+template <class C>
+__host__ __device__ constexpr int setup_barrier_threads() {
+    return kSetupWarps * 32 + 32 + (C::SCR_CONV ? kXThreads : 0);
+}
 
 // v = hi + lo with hi = v truncated to bf16 (its top 16 bits, a byte permute)
 // and lo = v - hi (exact in fp32) rounded to bf16: about 16 significant bits in
@@ -376,7 +387,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         fence_proxy_async_smem();  // the scratch is read before TMA writes reuse it
         tc_fence_before();
-        named_barrier_sync(3, kSetupThreads + 32);  // with the TMA producer (warp 0)
+        named_barrier_sync(3, setup_barrier_threads<C>());  // with the TMA producer (and the split warps)
         tc_fence_after();
     }
     // Buffer hand-offs from the tensor pipe are commits by the MMA warp: stage 1
@@ -401,8 +412,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int64_t g0 = int64_t(blockIdx.x) * C::GB;
         const int64_t gstep = int64_t(gridDim.x) * C::GB;
         for (int64_t j = 0; j < nb; ++j, g0 += gstep, rx.next(C::SX)) {
-            if (!setup_seen && j == C::SX - C::NSCR) {
-                named_barrier_sync(3, kSetupWarps * 32 + 32);
+            if (!setup_seen && j == C::SX - C::NSCR_RAW) {
+                named_barrier_sync(3, setup_barrier_threads<C>());
                 setup_seen = true;
             }
             const bool ok = wait_bounded(bar(C::EMPTY + rx.idx), rx.phase ^ 1u, s_abort, kSiteProducer,
@@ -426,7 +437,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             __syncwarp();
             ++issued;
         }
-        if (!setup_seen) named_barrier_sync(3, kSetupWarps * 32 + 32);  // fewer batches than free stages
+        if (!setup_seen) named_barrier_sync(3, setup_barrier_threads<C>());  // fewer batches than free stages
         // Drain: every load issued has landed (the slots' last phases completed).
         wait_bounded(bar(C::FACT), 0u, s_abort, kSiteDrain, kWaitLimitNs, true);
         Ring rd;
@@ -475,7 +486,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
                             const uint32_t b = (pass ? bl_lo : bl_hi) + koff1(kk);
-                            const uint32_t id1 = idesc1;
+                            // n1 > 64 with cinv: the lo tile holds -lo
+                            const uint32_t id1 = (SCALED && N1 > 64 && pass == 1) ? (idesc1 | (1u << 14)) : idesc1;
                             if (C::A1_TMEM) {
                                 if ((pass | kk) != 0)
                                     mma_ts_split<1>(d1, tmem + 8 * kk, b, kSdescSw128Hi, id1);
@@ -542,7 +554,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
     } else if (xsplit_index(warp) >= 0) {
         // ---------------- x' = x * cinv -> hi / lo bf16 tiles ----------------
-        if (SCALED) {
+        if constexpr (SCALED && N1 > 64) {
+            // n1 > 64: 5 to 8 units per thread, too many to keep their cinv values in
+            // registers; each unit's eight cinv values come through the read-only
+            // cache (the whole vector, n fp32, stays in L1/L2).  x' = x * cinv in fp32
+            // (one packed multiply per pair), then hi = x' truncated to bf16 and -lo =
+            // hi - x' by a mixed bf16/fp32 subtraction, rounded to bf16; the lo tile
+            // holds -lo, which stage 1 multiplies with the MMA's negate-B bit.
+            const int t = 32 * xsplit_index(warp) + lane;  // 0 .. kXThreads - 1
+            constexpr int UPT = 16 * N1 / kXThreads;       // units per thread per token
+            // the lo-half stages may hold the factor scratch until the setup is done
+            if constexpr (C::SCR_CONV) named_barrier_sync(3, setup_barrier_threads<C>());
+            static_assert(C::GB == 1, "one group per batch for n1 > 64");
+            Ring rx, rc;
+            for (int64_t j = 0; j < nb; ++j, rx.next(C::SX), rc.next(C::SC)) {
+                bool ok = wait_bounded(bar(C::FULL + rx.idx), rx.phase, s_abort, kSiteXSplit, kWaitLimitNs, false);
+                ok = ok && wait_bounded(bar(C::CEMPTY + rc.idx), rc.phase ^ 1u, s_abort, kSiteXSplit,
+                                        kWaitLimitNs, false);
+                if (!__all_sync(0xffffffffu, ok)) break;  // the warp leaves together
+                unsigned char *raw = smem + C::OFF_RAW + rx.idx * C::XTILE;  // x in, hi half out
+                unsigned char *lo = smem + C::OFF_CONV + rc.idx * C::XTILE;
+#pragma unroll 2
+                for (int u = 0; u < UPT; ++u) {
+                    // unit e: row r of chunk c, 16-byte column up of the swizzled tile,
+                    // i.e. channels r n2 + b0 .. + 7
+                    const int e = t + kXThreads * u;
+                    const int c = e / (8 * N1), rem = e % (8 * N1), r = rem >> 3, up = rem & 7;
+                    const int b0 = (N2 == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
+                    const float4 ca = __ldg(reinterpret_cast<const float4 *>(cinv + r * N2 + b0));
+                    const float4 cb = __ldg(reinterpret_cast<const float4 *>(cinv + r * N2 + b0 + 4));
+                    const int off = c * C::CHUNK + rem * 16;
+                    const uint4 in = *reinterpret_cast<const uint4 *>(raw + off);
+                    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+                    const float cv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+                    uint32_t oh[4], ol[4];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const uint64_t xp = uint64_t(w[p] << 16) | (uint64_t(w[p] & 0xFFFF0000u) << 32);
+                        const uint64_t cp = uint64_t(__float_as_uint(cv[2 * p])) |
+                                            (uint64_t(__float_as_uint(cv[2 * p + 1])) << 32);
+                        const uint64_t v = f32x2_mul(xp, cp);
+                        split_pair_neg(uint32_t(v), uint32_t(v >> 32), oh[p], ol[p]);
+                    }
+                    *reinterpret_cast<uint4 *>(raw + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+                    *reinterpret_cast<uint4 *>(lo + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(bar(C::CFULL + rc.idx));
+            }
+        } else if constexpr (SCALED) {
             const int t = 32 * xsplit_index(warp) + lane;  // 0 .. kXThreads - 1
             constexpr int UPT = 16 * N1 / kXThreads;             // units per thread per group
             // thread t handles unit e = t + kXThreads u (u < UPT) of every group of the
@@ -861,14 +921,12 @@ cudaError_t dispatch_n1(const LaunchArgs &a) {
     case 64: return launch_inst<64, N2, SCALED>(a);
     default: break;
     }
-    if constexpr (!SCALED) {
-        switch (a.n1) {
-        case 80: return launch_inst<80, N2, false>(a);
-        case 96: return launch_inst<96, N2, false>(a);
-        case 112: return launch_inst<112, N2, false>(a);
-        case 128: return launch_inst<128, N2, false>(a);
-        default: break;
-        }
+    switch (a.n1) {
+    case 80: return launch_inst<80, N2, SCALED>(a);
+    case 96: return launch_inst<96, N2, SCALED>(a);
+    case 112: return launch_inst<112, N2, SCALED>(a);
+    case 128: return launch_inst<128, N2, SCALED>(a);
+    default: break;
     }
     return cudaErrorNotSupported;
 }
@@ -889,9 +947,9 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 bool tc05_supports(int n1, int n2, bool scaled) {
+    (void)scaled;
     if (n2 != 64 && n2 != 128) return false;
-    if (n1 < 16 || n1 > 128 || n1 % 16) return false;
-    return !scaled || n1 <= 64;
+    return n1 >= 16 && n1 <= 128 && n1 % 16 == 0;
 }
 
 cudaError_t launch_tc05(const LaunchArgs &a) {

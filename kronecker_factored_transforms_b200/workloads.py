@@ -117,6 +117,11 @@ CONFIGS = {
     "mlp14336": dict(T=4096, n1=112, n2=128, seed=3, alpha=0.9, factors="orthogonal",
                      x_kind="relu_gated", outliers=("frac", 0.005, 40.0), pivot=None,
                      scaled=False),
+    # mlp14336 with a per-channel smoothing factor c ~ logU[0.5, 2] (cinv =
+    # 1 / c folded into the transform, as in hidden8192); seed 7.
+    "mlp14336_cinv": dict(T=4096, n1=112, n2=128, seed=7, alpha=0.9, factors="orthogonal",
+                          x_kind="relu_gated", outliers=("frac", 0.005, 40.0), pivot=None,
+                          scaled=True),
     # n=4096 (64x64) at T in SWEEP_T; N(0,1) + 1% x30; orthogonal;
     # alpha = 0.9; seed 4.
     "sweep4096": dict(T=1024, n1=64, n2=64, seed=4, alpha=0.9, factors="orthogonal",

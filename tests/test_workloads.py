@@ -20,8 +20,8 @@ def test_bf16_cast_is_round_to_nearest_even():
     np.testing.assert_array_equal(bf16_bits_to_f32(ours), torch.from_numpy(a).to(torch.bfloat16).float().numpy())
 
 
-@pytest.mark.parametrize("name", ["tiny", "llama7b_hidden", "hidden8192", "mlp14336", "sweep4096", "ffn28672",
-                                  "square65536"])
+@pytest.mark.parametrize("name", ["tiny", "llama7b_hidden", "hidden8192", "mlp14336", "mlp14336_cinv",
+                                  "sweep4096", "ffn28672", "square65536"])
 def test_shapes_and_reproducibility(name):
     a = make_workload(name, rows=8)
     b = make_workload(name, rows=8)
