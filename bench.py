@@ -51,6 +51,7 @@ KERNEL_SOURCES = ["kronecker_factored_transforms_b200/csrc/kq_fused.cu",
 
 
 def parse():
+    global WORKLOAD
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
@@ -61,6 +62,9 @@ def parse():
                          "of packed codes that consumes it (M = N = K = 8192); two_stage: the path for "
                          "factors above 128 (--two-stage-config); headwise: the per-head key/value "
                          "transform + INT4 (8192 tokens x 32 heads x 128)")
+    ap.add_argument("--config", choices=["hidden8192", "llama7b_hidden", "mlp14336", "mlp14336_cinv", "sweep4096"],
+                    default=WORKLOAD,
+                    help="configuration of the transform workload (both arms); the default is the headline one")
     ap.add_argument("--two-stage-config", choices=["square65536", "ffn28672"], default="square65536")
     ap.add_argument("--headwise-format", choices=["int4", "nvfp4"], default="int4",
                     help="rows of the headwise workload: INT4 with one scale, or NVFP4 (E2M1, an E4M3 scale per 16)")
@@ -75,12 +79,14 @@ def parse():
     ap.add_argument("--tokens", type=int, default=None,
                     help="token count of the transform workload instead of its own (profiling runs on a "
                          "smaller case; the JSON line's config names the count used)")
-    return ap.parse_args()
+    args = ap.parse_args()
+    WORKLOAD = args.config
+    return args
 
 
 def config_dict(w, extra=None):
-    d = {"workload": "%s: T=%d tokens/GPU, n=%d (n1=%d, n2=%d), cinv per channel, alpha=%g"
-         % (WORKLOAD, w.T, w.n, w.n1, w.n2, w.alpha),
+    d = {"workload": "%s: T=%d tokens/GPU, n=%d (n1=%d, n2=%d), %s, alpha=%g"
+         % (WORKLOAD, w.T, w.n, w.n1, w.n2, "cinv per channel" if w.cinv is not None else "no cinv", w.alpha),
          "T": w.T, "n": w.n, "n1": w.n1, "n2": w.n2, "alpha": w.alpha, "cinv": w.cinv is not None}
     if extra:
         d.update(extra)

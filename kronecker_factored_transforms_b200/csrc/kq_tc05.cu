@@ -555,17 +555,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (xsplit_index(warp) >= 0) {
         // ---------------- x' = x * cinv -> hi / lo bf16 tiles ----------------
         if constexpr (SCALED && N1 > 64) {
-            // n1 > 64: 5 to 8 units per thread, too many to keep their cinv values in
-            // registers; each unit's eight cinv values come through the read-only
-            // cache (the whole vector, n fp32, stays in L1/L2).  x' = x * cinv in fp32
-            // (one packed multiply per pair), then hi = x' truncated to bf16 and -lo =
-            // hi - x' by a mixed bf16/fp32 subtraction, rounded to bf16; the lo tile
-            // holds -lo, which stage 1 multiplies with the MMA's negate-B bit.
+            // n1 > 64: 5 to 8 units per thread.  The first UR units keep their cinv in
+            // registers as two bf16 values, cinv = ch + cl (RN(cinv) and RN of the
+            // rest): hi = RN(x ch), -lo = RN(-x cl + RN(-x ch + hi)), three packed bf16
+            // operations per pair.  The other units read their cinv through the
+            // read-only cache (UG x 8 KB per CTA, which stays in L1), form x' = x cinv
+            // in fp32 (one packed multiply per pair) and split it into hi = x'
+            // truncated to bf16 and -lo = RN(hi - x') (a mixed bf16/fp32 subtraction).
+            // Either way the lo tile holds -lo, which stage 1 multiplies with the
+            // MMA's negate-B bit; hi + lo is x cinv to about 2^-14 relative.
             const int t = 32 * xsplit_index(warp) + lane;  // 0 .. kXThreads - 1
             constexpr int UPT = 16 * N1 / kXThreads;       // units per thread per token
+            constexpr int UR = N1 == 96 ? 3 : 4, UG = UPT - UR;  // register units, cached units
+            static_assert(C::GB == 1 && UG >= 1 && UG <= 5, "one group per batch for n1 > 64");
+            // unit e = t + kXThreads u: row r of chunk c, 16-byte column up of the
+            // swizzled tile, i.e. channels r n2 + b0 .. + 7
+            auto chan0 = [&](int u) {
+                const int e = t + kXThreads * u;
+                const int c = e / (8 * N1), rem = e % (8 * N1), r = rem >> 3, up = rem & 7;
+                return r * N2 + (N2 == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
+            };
+            auto tile_off = [&](int u) {
+                const int e = t + kXThreads * u;
+                return (e / (8 * N1)) * C::CHUNK + (e % (8 * N1)) * 16;
+            };
+            uint32_t ch[UR][4], ncl[UR][4];
+            {
+                float4 ca[UR], cb[UR];  // every load first
+#pragma unroll
+                for (int u = 0; u < UR; ++u) {
+                    ca[u] = __ldg(reinterpret_cast<const float4 *>(cinv + chan0(u)));
+                    cb[u] = __ldg(reinterpret_cast<const float4 *>(cinv + chan0(u) + 4));
+                }
+#pragma unroll
+                for (int u = 0; u < UR; ++u) {
+                    const float cv[8] = {ca[u].x, ca[u].y, ca[u].z, ca[u].w, cb[u].x, cb[u].y, cb[u].z, cb[u].w};
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const float c0 = cv[2 * p], c1 = cv[2 * p + 1];
+                        ch[u][p] = pack_bf16x2(c0, c1);
+                        ncl[u][p] = bf16x2_neg(pack_bf16x2(c0 - __uint_as_float(ch[u][p] << 16),
+                                                           c1 - __uint_as_float(ch[u][p] & 0xFFFF0000u)));
+                    }
+                }
+            }
             // the lo-half stages may hold the factor scratch until the setup is done
             if constexpr (C::SCR_CONV) named_barrier_sync(3, setup_barrier_threads<C>());
-            static_assert(C::GB == 1, "one group per batch for n1 > 64");
             Ring rx, rc;
             for (int64_t j = 0; j < nb; ++j, rx.next(C::SX), rc.next(C::SC)) {
                 bool ok = wait_bounded(bar(C::FULL + rx.idx), rx.phase, s_abort, kSiteXSplit, kWaitLimitNs, false);
@@ -574,19 +609,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!__all_sync(0xffffffffu, ok)) break;  // the warp leaves together
                 unsigned char *raw = smem + C::OFF_RAW + rx.idx * C::XTILE;  // x in, hi half out
                 unsigned char *lo = smem + C::OFF_CONV + rc.idx * C::XTILE;
-#pragma unroll 2
-                for (int u = 0; u < UPT; ++u) {
-                    // unit e: row r of chunk c, 16-byte column up of the swizzled tile,
-                    // i.e. channels r n2 + b0 .. + 7
-                    const int e = t + kXThreads * u;
-                    const int c = e / (8 * N1), rem = e % (8 * N1), r = rem >> 3, up = rem & 7;
-                    const int b0 = (N2 == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
-                    const float4 ca = __ldg(reinterpret_cast<const float4 *>(cinv + r * N2 + b0));
-                    const float4 cb = __ldg(reinterpret_cast<const float4 *>(cinv + r * N2 + b0 + 4));
-                    const int off = c * C::CHUNK + rem * 16;
+                // the first cached units' loads are in flight during the register units
+                constexpr int PF = UG < 2 ? UG : 2;
+                float4 ga[UG], gb[UG];
+#pragma unroll
+                for (int g = 0; g < PF; ++g) {
+                    ga[g] = __ldg(reinterpret_cast<const float4 *>(cinv + chan0(UR + g)));
+                    gb[g] = __ldg(reinterpret_cast<const float4 *>(cinv + chan0(UR + g) + 4));
+                }
+#pragma unroll
+                for (int u = 0; u < UR; ++u) {
+                    const int off = tile_off(u);
                     const uint4 in = *reinterpret_cast<const uint4 *>(raw + off);
                     const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-                    const float cv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+                    uint32_t oh[4], ol[4];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        oh[p] = bf16x2_mul(w[p], ch[u][p]);
+                        const uint32_t nrest = bf16x2_fma(w[p], bf16x2_neg(ch[u][p]), oh[p]);
+                        ol[p] = bf16x2_fma(w[p], ncl[u][p], nrest);
+                    }
+                    *reinterpret_cast<uint4 *>(raw + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+                    *reinterpret_cast<uint4 *>(lo + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+                }
+#pragma unroll
+                for (int g = 0; g < UG; ++g) {
+                    if (g + PF < UG) {  // keep PF loads in flight
+                        ga[g + PF] = __ldg(reinterpret_cast<const float4 *>(cinv + chan0(UR + g + PF)));
+                        gb[g + PF] = __ldg(reinterpret_cast<const float4 *>(cinv + chan0(UR + g + PF) + 4));
+                    }
+                    const int off = tile_off(UR + g);
+                    const uint4 in = *reinterpret_cast<const uint4 *>(raw + off);
+                    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+                    const float cv[8] = {ga[g].x, ga[g].y, ga[g].z, ga[g].w, gb[g].x, gb[g].y, gb[g].z, gb[g].w};
                     uint32_t oh[4], ol[4];
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
