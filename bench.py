@@ -66,6 +66,8 @@ def parse():
                     default=WORKLOAD,
                     help="configuration of the transform workload (both arms); the default is the headline one")
     ap.add_argument("--two-stage-config", choices=["square65536", "ffn28672"], default="square65536")
+    ap.add_argument("--gemm-out", choices=["fp32", "bf16"], default="fp32",
+                    help="output dtype of the gemm workload (kq_w4a4_gemm or kq_w4a4_gemm_bf16)")
     ap.add_argument("--headwise-format", choices=["int4", "nvfp4"], default="int4",
                     help="rows of the headwise workload: INT4 with one scale, or NVFP4 (E2M1, an E4M3 scale per 16)")
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -295,8 +297,9 @@ class ClockSampler:
 
 def run_gemm(args):
     """The W4A4 product y = sx sw (qx qw^T) of a hidden-8192 layer: M tokens x
-    N output channels x K = n, packed INT4 codes in, fp32 out.  One step is one
-    kq_w4a4_gemm call; ops = 2 M N K.  Single GPU only."""
+    N output channels x K = n, packed INT4 codes in, fp32 (or bf16) out.  One
+    step is one kq_w4a4_gemm (kq_w4a4_gemm_bf16) call; ops = 2 M N K.  Single
+    GPU only."""
     import torch
     from kronecker_factored_transforms_b200 import _lib
     M = N = K = 8192
@@ -306,17 +309,19 @@ def run_gemm(args):
     qw = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
     sx = torch.rand(M, device=dev, generator=g)
     sw = torch.rand(N, device=dev, generator=g)
-    y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    bf16 = args.gemm_out == "bf16"
+    y = torch.empty((M, N), dtype=torch.bfloat16 if bf16 else torch.float32, device=dev)
+    gemm = _lib.kq_w4a4_gemm_bf16 if bf16 else _lib.kq_w4a4_gemm
     stream = torch.cuda.current_stream(dev)
     for _ in range(max(3, args.warmup)):
-        _lib.kq_w4a4_gemm(qx, sx, qw, sw, y, M, N, K, stream=stream.cuda_stream)
+        gemm(qx, sx, qw, sw, y, M, N, K, stream=stream.cuda_stream)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(0)
     with sampler:
         e0.record(stream)
         for _ in range(args.steps):
-            _lib.kq_w4a4_gemm(qx, sx, qw, sw, y, M, N, K, stream=stream.cuda_stream)
+            gemm(qx, sx, qw, sw, y, M, N, K, stream=stream.cuda_stream)
         e1.record(stream)
         torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1) / args.steps
@@ -326,8 +331,9 @@ def run_gemm(args):
     line = {"metric": "TOPS of the W4A4 product of packed INT4 codes (M = N = K = 8192)", "value": tops,
             "unit": "TOPS", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4 (int8 MMA)",
-            "data": "synthetic", "config": {"workload": "w4a4 gemm M=N=K=8192, random codes and scales",
-                                             "M": M, "N": N, "K": K},
+            "data": "synthetic", "config": {"workload": "w4a4 gemm M=N=K=8192, random codes and scales, %s out"
+                                                         % args.gemm_out, "M": M, "N": N, "K": K,
+                                             "out": args.gemm_out},
             "roofline": {"bound": "tensor", "achieved": tops, "peak": int8_peak, "unit": "TOP/s",
                          "frac": tops / int8_peak, "traffic": None,
                          "peak_source": "2 x %s bf16 TF/s (int8 dense rate)" % kind},

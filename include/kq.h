@@ -135,6 +135,17 @@ kq_status kq_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, co
                        int64_t M, int64_t N, int64_t K, kq_stream_t stream);
 
 /*
+ * kq_w4a4_gemm_bf16 -- kq_w4a4_gemm with a bf16 output (the next layer's
+ * activation dtype): y [M, N] device bf16 bits, row-major, 2-byte aligned,
+ * written; each element is kq_w4a4_gemm's fp32 value rounded to the nearest
+ * bf16 (ties to even).  Same arguments, checks and status codes otherwise.
+ * Writing half the bytes is what a large product needs: at M = N = K = 8192
+ * the fp32 output is the larger part of its memory traffic.
+ */
+kq_status kq_w4a4_gemm_bf16(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw, uint16_t *y,
+                            int64_t M, int64_t N, int64_t K, kq_stream_t stream);
+
+/*
  * kq_headwise_transform_quant -- the per-head transform of the key / value
  * cache (FlatQuant page: P_h and P_v keep their full per-head shape; keys and
  * values are transformed per head and quantised before storage).  For every

@@ -42,12 +42,13 @@ def _load() -> ctypes.CDLL:
     lib.kq_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
     lib.kq_selftest_bounded_wait.argtypes = [I64, P]
     lib.kq_w4a4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P]
+    lib.kq_w4a4_gemm_bf16.argtypes = [P, P, P, P, P, I64, I64, I64, P]
     lib.kq_headwise_transform_quant.argtypes = [P, P, F32, P, P, I64, I32, I32, P]
     lib.kq_transform_quant_two_stage.argtypes = [P, P, P, P, F32, P, P, P, ctypes.c_uint64, I64, I32, I32, P]
     lib.kq_transform_quant_two_stage_static.argtypes = [P, P, P, P, F32, P, P, I64, I32, I32, P]
     lib.kq_headwise_transform_quant_nvfp4.argtypes = [P, P, P, P, P, I64, I32, I32, P]
     for f in (lib.kq_transform_quant, lib.kq_transform, lib.kq_dequant_inverse, lib.kq_device_error,
-              lib.kq_selftest_bounded_wait, lib.kq_w4a4_gemm, lib.kq_headwise_transform_quant,
+              lib.kq_selftest_bounded_wait, lib.kq_w4a4_gemm, lib.kq_w4a4_gemm_bf16, lib.kq_headwise_transform_quant,
               lib.kq_transform_quant_two_stage, lib.kq_transform_quant_two_stage_static,
               lib.kq_headwise_transform_quant_nvfp4):
         f.restype = ctypes.c_int
@@ -68,6 +69,7 @@ lib = _load()
 
 EXPORTED = ("kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_device_error",
             "kq_selftest_bounded_wait", "kq_status_string", "kq_kernel_name", "kq_kernel_for", "kq_version", "kq_w4a4_gemm",
+            "kq_w4a4_gemm_bf16",
             "kq_headwise_transform_quant", "kq_transform_quant_two_stage", "kq_two_stage_workspace_bytes",
             "kq_transform_quant_two_stage_static", "kq_headwise_transform_quant_nvfp4")
 
@@ -141,6 +143,12 @@ def kq_w4a4_gemm(qx, sx, qw, sw, y, M: int, N: int, K: int, stream=None) -> None
     _check("kq_w4a4_gemm",
            lib.kq_w4a4_gemm(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), _ptr(y), int(M), int(N), int(K),
                             _stream(stream)))
+
+
+def kq_w4a4_gemm_bf16(qx, sx, qw, sw, y, M: int, N: int, K: int, stream=None) -> None:
+    _check("kq_w4a4_gemm_bf16",
+           lib.kq_w4a4_gemm_bf16(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), _ptr(y), int(M), int(N), int(K),
+                                 _stream(stream)))
 
 
 def kq_transform(x, P1, P2, cinv, y_out, T: int, n1: int, n2: int, stream=None) -> None:

@@ -185,26 +185,39 @@ kq_status kq_dequant_inverse(const uint8_t *q, const float *scale, const float *
     return err == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;
 }
 
-kq_status kq_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw, float *y,
-                       int64_t M, int64_t N, int64_t K, kq_stream_t stream) {
+namespace {
+// The checks and the launch of both W4A4 entries; `ob` = output bytes per element.
+kq_status w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw, void *y, int ob,
+                    int64_t M, int64_t N, int64_t K, kq_stream_t stream) {
     if (M < 0 || N < 0 || K < 128 || K > 262144 || K % 128 != 0) return KQ_ERR_SHAPE;
     if (M > int64_t(65535) * 128) return KQ_ERR_SHAPE;  // grid rows
     if (M == 0 || N == 0) return KQ_OK;
     if (M > INT64_MAX / N / 4) return KQ_ERR_SHAPE;
     if (!qx || !sx || !qw || !sw || !y) return KQ_ERR_NULL;
-    if (!aligned(qx, 16) || !aligned(qw, 16) || !aligned(sx, 4) || !aligned(sw, 4) || !aligned(y, 4))
+    if (!aligned(qx, 16) || !aligned(qw, 16) || !aligned(sx, 4) || !aligned(sw, 4) || !aligned(y, uintptr_t(ob)))
         return KQ_ERR_ALIGN;
     const Range in[4] = {range_of(qx, uint64_t(M) * uint64_t(K) / 2), range_of(sx, uint64_t(M) * 4),
                          range_of(qw, uint64_t(N) * uint64_t(K) / 2), range_of(sw, uint64_t(N) * 4)};
-    const Range ry = range_of(y, uint64_t(M) * uint64_t(N) * 4);
+    const Range ry = range_of(y, uint64_t(M) * uint64_t(N) * uint64_t(ob));
     for (const Range &r : in)
         if (overlap(r, ry)) return KQ_ERR_ARG;
     DeviceInfo info;
     kq_status st = device_info(info);
     if (st != KQ_OK) return st;
-    cudaError_t err = kq::launch_w4a4_gemm(qx, sx, qw, sw, y, M, N, K, info.device,
+    cudaError_t err = kq::launch_w4a4_gemm(qx, sx, qw, sw, y, ob == 2, M, N, K, info.device,
                                            reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? KQ_OK : KQ_ERR_CUDA;
+}
+}  // namespace
+
+kq_status kq_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw, float *y,
+                       int64_t M, int64_t N, int64_t K, kq_stream_t stream) {
+    return w4a4_gemm(qx, sx, qw, sw, y, 4, M, N, K, stream);
+}
+
+kq_status kq_w4a4_gemm_bf16(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw, uint16_t *y,
+                            int64_t M, int64_t N, int64_t K, kq_stream_t stream) {
+    return w4a4_gemm(qx, sx, qw, sw, y, 2, M, N, K, stream);
 }
 
 kq_status kq_headwise_transform_quant(const uint16_t *x, const uint16_t *Ph, float alpha, uint8_t *q_out,

@@ -5,7 +5,9 @@
 //
 // qx [M, K/2] and qw [N, K/2] hold two's-complement INT4 codes, element 2k in
 // the low nibble of byte k (the layout kq_transform_quant writes), sx [M] and
-// sw [N] the per-token and per-output-channel fp32 scales, y [M, N] fp32.
+// sw [N] the per-token and per-output-channel fp32 scales, y [M, N] fp32, or
+// bf16 (the fp32 value rounded to nearest even), which halves the output bytes
+// that dominate the traffic of a large product.
 //
 // The 5th-generation tensor cores have no 4-bit integer kind, so each 128-code
 // K chunk goes: packed tiles by TMA -> eight expander warps widen every code q
@@ -79,9 +81,39 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
 // Byte offset of the 16-byte chunk `c` of row `r` in a 128B-swizzled K-major tile.
 __device__ __forceinline__ uint32_t sw128_chunk(int r, int c) { return uint32_t(r * 128 + ((c ^ (r & 7)) << 4)); }
 
+// y[n .. n + 3] of one row: fp32 as is, or rounded to bf16 (nearest even);
+// one 16-byte (fp32) or 8-byte (bf16) store where `vec` allows it.
+template <bool BF16>
+__device__ __forceinline__ void store_out4(void *yrow, int64_t n, int64_t N, bool vec, const float (&r4)[4]) {
+    if constexpr (BF16) {
+        uint16_t *p = static_cast<uint16_t *>(yrow) + n;
+        const __nv_bfloat162 a = __floats2bfloat162_rn(r4[0], r4[1]), b = __floats2bfloat162_rn(r4[2], r4[3]);
+        if (vec && n + 3 < N) {
+            *reinterpret_cast<uint2 *>(p) = make_uint2(*reinterpret_cast<const uint32_t *>(&a),
+                                                       *reinterpret_cast<const uint32_t *>(&b));
+        } else {
+            const uint16_t h[4] = {__bfloat16_as_ushort(a.x), __bfloat16_as_ushort(a.y), __bfloat16_as_ushort(b.x),
+                                   __bfloat16_as_ushort(b.y)};
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                if (n + t < N) p[t] = h[t];
+        }
+    } else {
+        float *p = static_cast<float *>(yrow) + n;
+        if (vec && n + 3 < N) {
+            *reinterpret_cast<float4 *>(p) = make_float4(r4[0], r4[1], r4[2], r4[3]);
+        } else {
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                if (n + t < N) p[t] = r4[t];
+        }
+    }
+}
+
+template <bool BF16>
 __global__ void __launch_bounds__(G_THREADS, 1)
     kq_w4a4_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                      const float *__restrict__ sx, const float *__restrict__ sw, float *__restrict__ y,
+                      const float *__restrict__ sx, const float *__restrict__ sw, void *__restrict__ y,
                       int64_t M, int64_t N, int64_t K, unsigned int *err) {
     extern __shared__ __align__(1024) unsigned char gsm_raw[];
     const uint32_t raw_addr = smem_u32(gsm_raw);
@@ -246,9 +278,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             const int q = warp & 3, h = (warp - XW0) >> 2;  // lane quarter, column half
             const int64_t m = m0 + 32 * q + lane;
             const float fx = m < M ? sx[m] : 0.0f;
-            float *yrow = y + (m < M ? m : 0) * N;
-            // 16-byte stores only where every row start is 16-byte aligned
-            const bool vec = (N % 4) == 0 && (reinterpret_cast<uintptr_t>(y) & 15) == 0;
+            constexpr int OB = BF16 ? 2 : 4;  // output bytes per element
+            void *yrow = static_cast<unsigned char *>(y) + (m < M ? m : 0) * N * OB;
+            // vector stores only where every row start is aligned for them
+            const bool vec = (N % 4) == 0 && (reinterpret_cast<uintptr_t>(y) & (4 * OB - 1)) == 0;
 #pragma unroll 1
             for (int c = 0; c < TN / 2 / 32; ++c) {
                 uint32_t a[32];
@@ -263,13 +296,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 #pragma unroll
                         for (int t = 0; t < 4; ++t)
                             r4[t] = (float(int(a[e + t]) >> 8) * fx) * (n + t < N ? sw[n + t] : 0.0f);
-                        if (vec && n + 3 < N) {
-                            *reinterpret_cast<float4 *>(yrow + n) = make_float4(r4[0], r4[1], r4[2], r4[3]);
-                        } else {
-#pragma unroll
-                            for (int t = 0; t < 4; ++t)
-                                if (n + t < N) yrow[n + t] = r4[t];
-                        }
+                        store_out4<BF16>(yrow, n, N, vec, r4);
                     }
                 }
             }
@@ -287,14 +314,17 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 
 }  // namespace
 
-cudaError_t launch_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw, float *y,
-                             int64_t M, int64_t N, int64_t K, int device, cudaStream_t stream) {
+cudaError_t launch_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw, void *y,
+                             bool bf16_out, int64_t M, int64_t N, int64_t K, int device, cudaStream_t stream) {
     static std::once_flag once[64];
     static cudaError_t attr_err[64];
     if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[device], [&] {
-        attr_err[device] = cudaFuncSetAttribute(kq_w4a4_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                G_SMEM);
+        attr_err[device] = cudaFuncSetAttribute(kq_w4a4_tc_kernel<false>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM);
+        if (attr_err[device] == cudaSuccess)
+            attr_err[device] = cudaFuncSetAttribute(kq_w4a4_tc_kernel<true>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM);
     });
     if (attr_err[device] != cudaSuccess) return attr_err[device];
     unsigned int *err = nullptr;
@@ -317,7 +347,10 @@ cudaError_t launch_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     const dim3 grid(unsigned((N + TN - 1) / TN), unsigned((M + TM - 1) / TM));
-    kq_w4a4_tc_kernel<<<grid, G_THREADS, G_SMEM, stream>>>(ta, tb, sx, sw, y, M, N, K, err);
+    if (bf16_out)
+        kq_w4a4_tc_kernel<true><<<grid, G_THREADS, G_SMEM, stream>>>(ta, tb, sx, sw, y, M, N, K, err);
+    else
+        kq_w4a4_tc_kernel<false><<<grid, G_THREADS, G_SMEM, stream>>>(ta, tb, sx, sw, y, M, N, K, err);
     return cudaGetLastError();
 }
 

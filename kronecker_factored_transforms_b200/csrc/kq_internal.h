@@ -53,8 +53,8 @@ cudaError_t launch_dequant_inverse(const uint8_t *q, const float *scale, const f
                                    int n1, int n2, cudaStream_t stream);
 
 // W4A4 product of packed INT4 codes: y = sx[m] sw[o] sum_k qx[m][k] qw[o][k].
-cudaError_t launch_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw, float *y,
-                             int64_t M, int64_t N, int64_t K, int device, cudaStream_t stream);
+cudaError_t launch_w4a4_gemm(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw, void *y,
+                             bool bf16_out, int64_t M, int64_t N, int64_t K, int device, cudaStream_t stream);
 
 // Per-head transform + INT4 per row: rows of head_dim (64 or 128) values.
 cudaError_t launch_rowwise(const uint16_t *x, const uint16_t *Ph, float alpha, uint8_t *q_out, float *scale_out,

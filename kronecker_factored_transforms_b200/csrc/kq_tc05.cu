@@ -336,33 +336,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
         }
         if (!C::A1_TMEM) {
-            // A1[(h, m)][(h', b)] = P2[b][lane_column(m)] if h == h' else 0, from
-            // 16-byte pieces of rows of P2 (loads first), 128B-swizzled K-major.
-            constexpr int PIECES = N2 * N2 / 8, PER = (PIECES + kSetupThreads - 1) / kSetupThreads;
-            uint4 v[PER];
+            // A1[(h, m)][(h', b)] = P2[b][lane_column(m)] if h == h' else 0, 128B-swizzled
+            // K-major, built like B2: a piece is one row l and eight consecutive k, eight
+            // loads (consecutive threads take consecutive l, i.e. 32 distinct columns
+            // of one row of P2) and one 16-byte store.
+            constexpr int PIECES = 128 * 16, PER = (PIECES + kSetupThreads - 1) / kSetupThreads;
+            uint32_t w[PER][4];
 #pragma unroll
             for (int u = 0; u < PER; ++u) {
                 const int c = st + u * kSetupThreads;
-                if (c < PIECES) v[u] = *reinterpret_cast<const uint4 *>(P2s + 8 * c);
+                const int l = c % 128, k0 = 8 * (c / 128);
+                const int h = l / N2, j = lane_column(l % N2), hk = k0 / N2, b0 = k0 % N2;
+                const bool on = c < PIECES && h == hk;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t lo = on ? P2s[(b0 + 2 * e) * N2 + j] : 0u;
+                    const uint32_t hi = on ? P2s[(b0 + 2 * e + 1) * N2 + j] : 0u;
+                    w[u][e] = lo | (hi << 16);
+                }
             }
 #pragma unroll
             for (int u = 0; u < PER; ++u) {
                 const int c = st + u * kSetupThreads;
                 if (c < PIECES) {
-                    const int b = (8 * c) / N2, j0 = (8 * c) % N2;
-                    const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        const int m = lane_of_column(j0 + t);
-#pragma unroll
-                        for (int h = 0; h < C::H; ++h)
-#pragma unroll
-                            for (int hk = 0; hk < C::H; ++hk) {
-                                const int l = h * N2 + m, k = hk * N2 + b;
-                                *reinterpret_cast<uint16_t *>(smem + C::OFF_A1 + (k >> 6) * 16384 + swz128(l, k & 63)) =
-                                    h == hk ? uint16_t(w[t >> 1] >> (16 * (t & 1))) : uint16_t(0);
-                            }
-                    }
+                    const int l = c % 128, k0 = 8 * (c / 128);
+                    *reinterpret_cast<uint4 *>(smem + C::OFF_A1 + (k0 >> 6) * 16384 + swz128(l, k0 & 63)) =
+                        make_uint4(w[u][0], w[u][1], w[u][2], w[u][3]);
                 }
             }
         }

@@ -29,7 +29,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for must in ("kq_transform_quant", "kq_transform", "kq_dequant_inverse", "kq_status_string",
-                 "kq_kernel_name", "kq_kernel_for", "kq_device_error", "kq_version", "kq_w4a4_gemm",
+                 "kq_kernel_name", "kq_kernel_for", "kq_device_error", "kq_version", "kq_w4a4_gemm", "kq_w4a4_gemm_bf16",
                  "kq_headwise_transform_quant", "kq_transform_quant_two_stage", "kq_two_stage_workspace_bytes",
                  "kq_headwise_transform_quant_nvfp4"):
         assert must in names

@@ -81,6 +81,55 @@ def test_gemm_full_size_sampled_rows(kq):
     _check(y[rows], oracle.w4a4_gemm(qx[rows], sx[rows], qw, sw))
 
 
+def _bf16_to_f64(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _f64_to_bf16_rne(a):
+    """Round fp64 values to bf16 (nearest, ties to even) through float32 with
+    a sticky bit, so that no double rounding changes a tie."""
+    f = a.astype(np.float32)
+    # float32 rounding may have created or broken a bf16 tie: fall back to exact
+    # comparison of both bf16 neighbours of the float32 value
+    b = f.view(np.uint32)
+    lo = (b & 0xFFFF0000).view(np.float32).astype(np.float64)
+    hi = ((b & 0xFFFF0000) + 0x10000).astype(np.uint32).view(np.float32).astype(np.float64)
+    dlo, dhi = np.abs(a - lo), np.abs(hi - a)
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (((b >> 16) & 1) == 1))
+    return np.where(pick_hi, ((b >> 16) + 1) & 0xFFFF, (b >> 16) & 0xFFFF).astype(np.uint16)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 128), (37, 53, 256), (129, 127, 384), (200, 300, 1024), (513, 65, 14336)])
+def test_gemm_bf16_output(kq, M, N, K):
+    """kq_w4a4_gemm_bf16 rounds the fp32 value to the nearest bf16: equal to the
+    oracle's fp64 product rounded to bf16, except (by one bf16 ulp) where the
+    fp64 value lies within the fp32 error (2^-22 relative) of a bf16 midpoint."""
+    rng = np.random.default_rng(M * 5 + N * 11 + K)
+    qx, qw = _codes(rng, M, K), _codes(rng, N, K)
+    sx = rng.uniform(1e-3, 2.0, M).astype(np.float32)
+    sw = rng.uniform(1e-3, 2.0, N).astype(np.float32)
+    PADH = 2048
+    buf = torch.full((M * N + 2 * PADH,), 0x7FC1, dtype=torch.int16, device="cuda")
+    y = buf[PADH:PADH + M * N]
+    kq.kq_w4a4_gemm_bf16(torch.from_numpy(qx).cuda(), torch.from_numpy(sx).cuda(), torch.from_numpy(qw).cuda(),
+                         torch.from_numpy(sw).cuda(), y, M, N, K)
+    torch.cuda.synchronize()
+    b = buf.cpu().numpy()
+    assert (b[:PADH] == 0x7FC1).all() and (b[PADH + M * N:] == 0x7FC1).all(), "write outside y"
+    got = y.cpu().numpy().view(np.uint16).reshape(M, N)
+    ref64 = oracle.w4a4_gemm(qx, sx, qw, sw)
+    want = _f64_to_bf16_rne(ref64)
+    differ = got != want
+    if differ.any():
+        # only where the exact value is within the fp32 error of a bf16 midpoint
+        v = ref64[differ]
+        f = v.astype(np.float32).view(np.uint32)
+        mid = ((f & 0xFFFF0000) | 0x8000).view(np.float32).astype(np.float64)
+        assert (np.abs(v - mid) <= 2.0 ** -22 * np.abs(v)).all(), "bf16 outputs off beyond a midpoint"
+        assert (np.abs(got[differ].astype(np.int32) - want[differ].astype(np.int32)) <= 1).all()
+    assert differ.mean() < 1e-3
+
+
 def test_layer_codes_through_the_gemm(kq):
     """Activation codes from kq_transform_quant and weight codes from the
     weight-side transform, multiplied by kq_w4a4_gemm, equal the oracle's product
