@@ -1,5 +1,8 @@
 // kq_fused.cu -- persistent fused Kronecker transform + INT4 kernel on the
-// 5th-generation tensor cores, pipelined per group of tokens.
+// 5th-generation tensor cores, pipelined per pair of token groups; the kernel
+// kq_transform_quant runs for short launches at n1 = 64 (at most 24 groups
+// per SM), where the batch-pipelined kernel of kq_tc05.cu spends a larger
+// share of the launch filling and draining its pipeline.
 //
 // Method (FlatQuant page, "Kronecker factorization", "Per-channel scaling and
 // learnable clipping" and "The fused kernel"): per token Y~ = P1^T X~ P2 with
@@ -11,36 +14,44 @@
 // the group's 128 output columns j (n2 = 64: two tokens, P2^T block-diagonal).
 // TMEM lane m of a token holds column lane_column(m) (kq_tile.cuh), so that
 // the epilogue thread of a 16x256b load holds four consecutive columns: two
-// whole bytes of every output row.
+// whole bytes of every output row.  A CTA takes its groups (dealt round-robin)
+// in pairs.
 //
-//   stage 1   D1[l][a] = sum_k A1[l][k] X[a][k]: A1 = P2^T (TMEM, resident),
-//             X = the group's x tile (K = 128; with cinv its x' = x o cinv hi
-//             and lo bf16 tiles, accumulated in two passes), M = 128, N = n1.
-//   convert   D1 (fp32) -> A2 = hi + lo bf16 pairs, in place in TMEM.
-//   stage 2   D2[l][i] = sum_a A2[l][a] P1[a][i] (A from TMEM, B = P1^T in
-//             shared memory; hi and lo passes), M = 128, N = n1.
+//   stage 1   D1[l][a] = sum_k A1[l][k] X[a][k] for both groups of a pair in
+//             one MMA (M = 128, N = 2 n1 = 128, K = 128): A1 = P2^T (TMEM,
+//             resident), X = the pair's x tile, or with cinv its x' = x o cinv
+//             as -hi and lo bf16 tiles accumulated in two passes (the -hi pass
+//             with the MMA's negate-B bit).
+//   convert   D1 (fp32) -> A2 = hi and -lo bf16 halves, in place in TMEM.
+//   stage 2   D2[l][i] = sum_a A2[l][a] P1[a][i] per group (A from TMEM, B =
+//             P1^T in shared memory; the -lo pass with negate-B), M = 128, N = n1.
 //   epilogue  absmax over the token's lanes, quantise, pack, 16-bit stores
 //             straight to global memory, one fp32 scale per token.
 //
-// TMEM: P2^T (64 columns), NA = 5 D1/A2 slots and ND = 2 D2 slots of n1
-// columns.  One MMA thread issues stage 1 of group j + L before stage 2 of
-// group j, so the conversion of a group overlaps the tensor work of the
-// groups around it and every slot is reused only long after the MMAs that
-// read it completed.
+// TMEM: P2^T (64 columns), two D1/A2 regions of 2 n1 columns (one pair each)
+// and three D2 slots of n1 columns (one per epilogue warpgroup).  Stage 1 of a
+// pair reuses its region only after stage 2 of the pair two back completed, so
+// the tensor pipe runs stage 1 of two pairs, then stage 2 of the two pairs
+// before them, and so on.
 //
 // x reaches the kernel in one of two ways.  Without cinv, TMA copies each
-// group's x tile (128-byte swizzle, the K-major B layout) into a ring of
-// shared-memory slots that stage 1 reads as is.  With cinv, eight warps load
-// the group's x with 16-byte global loads (prefetched into L2 a few groups
-// ahead), form x' = x o cinv as hi + lo bf16 in registers and store the two
-// swizzled tiles; the raw x tile never passes through shared memory.
+// pair's x tile (128-byte swizzle, the K-major B layout) into a ring of
+// shared-memory slots that stage 1 reads as is.  With cinv, the split warps
+// load x with 16-byte global loads (prefetched into L2 a few pairs ahead by
+// warp 0), form x' = x o cinv as -hi + lo bf16 in registers (three packed bf16
+// operations per pair of values, cinv held in registers as two bf16 values)
+// and store the two swizzled tiles; the raw x tile never passes through shared
+// memory.
 //
-// Warp roles (24 warps): 0 factor copies, then (without cinv) the TMA
-// producer | 1 TMEM allocation and MMA issue | 2-3 set-up only | 4-11 x'
-// split (cinv) | 12-15 D1 -> A2 conversion | 16-19 and 20-23 two epilogue
-// warpgroups on alternate groups (each with its own D2 slot).  Every mbarrier
-// wait is bounded: after about a second it ORs a site bit into the device
-// status word, raises a CTA-wide abort flag and the roles drain and exit.
+// Warp roles (32 warps, at most 64 registers per thread): 0 factor copies,
+// then the TMA producer (without cinv) or the L2 prefetch (with cinv) | 1
+// TMEM allocation and stage-1 MMA issue | 3 stage-2 MMA issue | 4-19 x' split
+// (cinv) and the D1 -> A2 conversion, running the split two pairs ahead of
+// the conversion | 20-31 three epilogue warpgroups on groups j with j % 3 ==
+// warpgroup | 2 idle.  Warps 4-11 and 20-31 build P2^T (TMEM) and P1^T (shared
+// memory) at start.  Every mbarrier wait is bounded: after about a second it
+// ORs a site bit into the device status word, raises a CTA-wide abort flag and
+// the roles drain and exit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -144,18 +155,16 @@ __device__ __forceinline__ void split_pair_neg(uint32_t v0, uint32_t v1, uint32_
     nlo = pack_bf16x2(n0, n1);
 }
 
-// round_half_even(y * inv) of two values at once, for |y * inv| < 2^22: adding
-// 1.5 * 2^23 (one packed fp32x2 multiply-add) leaves the rounded integer in the
-// low mantissa bits (bit pattern 0x4B400000 + k); an integer multiply-add with
-// `one` (== 1, read at run time) removes the offset.
+// round_half_even(y * inv) as an int, for |y * inv| < 2^22: adding 1.5 * 2^23
+// leaves the rounded integer in the low mantissa bits (bit pattern 0x4B400000
+// + k); an integer multiply-add with `one` (== 1, read at run time) removes
+// the offset beside the floating-point work.
 constexpr uint32_t kFMagicBits = 0x4B400000u;  // 1.5 * 2^23
-__device__ __forceinline__ void round_code2(uint32_t y0, uint32_t y1, uint64_t inv2, int one, int &k0, int &k1) {
-    const uint64_t y = uint64_t(y0) | (uint64_t(y1) << 32);
-    const uint64_t magic = (uint64_t(kFMagicBits) << 32) | kFMagicBits;
-    uint64_t b;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(b) : "l"(y), "l"(inv2), "l"(magic));
-    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k0) : "r"(uint32_t(b)), "r"(one), "r"(-int(kFMagicBits)));
-    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k1) : "r"(uint32_t(b >> 32)), "r"(one), "r"(-int(kFMagicBits)));
+__device__ __forceinline__ int round_code(uint32_t ybits, float inv, int one) {
+    const uint32_t b = __float_as_uint(fmaf(__uint_as_float(ybits), inv, 12582912.0f));
+    int k;
+    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k) : "r"(b), "r"(one), "r"(-int(kFMagicBits)));
+    return k;
 }
 
 template <int N1, int N2, bool SCALED>
@@ -221,7 +230,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
         mbar_init(bar(C::SETUP), kSetupArrivals);
         mbar_init(bar(C::TEARDOWN), 2);
         *s_abort = 0;
-        *reinterpret_cast<int *>(smem + C::OFF_MISC + 8) = 1;  // `one` of round_code2
+        *reinterpret_cast<int *>(smem + C::OFF_MISC + 8) = 1;  // `one` of round_code
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0 && !SCALED) prefetch_tensormap(&tmap_x);
@@ -630,7 +639,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
             // the exact quotients by a few ulps, far inside the rounding-boundary window
             const float s = alpha * m * (1.0f / 7.0f);
             const float inv = s > 0.0f ? fminf(__fdividef(1.0f, s), 3.0e38f) : 0.0f;
-            const uint64_t inv2 = (uint64_t(__float_as_uint(inv)) << 32) | __float_as_uint(inv);
             const int64_t tok = group_of(j) * C::H + tok_h;
             const bool live = tok < T;
             // this thread's two bytes of rows i = 16 c0 + 8 rep + 2 qq + d of its token
@@ -652,10 +660,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
                         // rows 16 c0 + 8 rep + 2 qq + d: columns 4 g8 + (0, 1) from half 0,
                         // + (2, 3) from half 1; even column in the low nibble
                         int ka[4], kb[4];
-                        round_code2(ra[4 * rep], ra[4 * rep + 1], inv2, one, ka[0], ka[1]);
-                        round_code2(ra[4 * rep + 2], ra[4 * rep + 3], inv2, one, ka[2], ka[3]);
-                        round_code2(rb[4 * rep], rb[4 * rep + 1], inv2, one, kb[0], kb[1]);
-                        round_code2(rb[4 * rep + 2], rb[4 * rep + 3], inv2, one, kb[2], kb[3]);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            ka[e] = round_code(ra[4 * rep + e], inv, one);
+                            kb[e] = round_code(rb[4 * rep + e], inv, one);
+                        }
 #pragma unroll
                         for (int d = 0; d < 2; ++d) {
                             const uint32_t wb = pack_s4x2(kb[2 + d], kb[d], 0u);

@@ -1,6 +1,8 @@
 // kq_tc05.cu -- persistent fused Kronecker transform + INT4 kernel on the
-// 5th-generation tensor cores (tcgen05.mma, accumulators in TMEM), plus the
-// device status word that its bounded waits report through.
+// 5th-generation tensor cores (tcgen05.mma, accumulators in TMEM), pipelined
+// per batch of token groups: the kernel kq_transform_quant runs for long
+// launches and for n1 != 64 (kq_fused.cu takes short launches at n1 = 64);
+// plus the device status word that the bounded waits report through.
 //
 // Method (FlatQuant page, "Kronecker factorization" and "The fused kernel"):
 // per token Y~ = P1^T X~ P2 with X~ the row-major n1 x n2 view of x * cinv,
@@ -19,14 +21,18 @@
 //                     A1 = block-diag over h of P2^T (rows permuted as above),
 //                     resident in TMEM (or shared memory for n1 > 96);
 //                     X  = the group's x tile straight from TMA (K = 128).
-//   convert (TMEM)    D1 fp32 -> A2 = hi + lo bf16, in place, chunk by chunk.
-//   stage 2 (TS MMA)  D2[l][i]  = sum_a A2[l][a] * P1[a][i]   (A from TMEM)
+//   convert (TMEM)    D1 fp32 -> A2 = hi and -lo bf16, in place, chunk by chunk
+//                     (hi = the top 16 bits, -lo = hi - D1 by one mixed
+//                     bf16/fp32 subtraction).
+//   stage 2 (TS MMA)  D2[l][i]  = sum_a A2[l][a] * P1[a][i]   (A from TMEM; the
+//                     -lo pass with the MMA's negate-B bit)
 //   epilogue          absmax over the token's lanes, quantise, pack into a
 //                     swizzled staging tile, one TMA store per group to HBM.
 // With cinv, the x' split warps turn each raw x tile into x' = x * cinv
 // split into a hi bf16 tile (written over x) and a lo bf16 tile; stage 1
-// then accumulates both.  TMEM holds P2^T, two D1/A2 regions (batches) and
-// three D2 regions (groups, n1 <= 64).
+// then accumulates both (for n1 > 64 the lo tile holds -lo and its pass
+// negates B).  TMEM holds P2^T, two D1/A2 regions (batches) and two or
+// three D2 regions (groups).
 //
 // Warp roles: 0 TMA producer | 1 TMEM allocator + stage-1 MMA issuer | 5
 // stage-2 MMA issuer | 2-4, 6-7, 20, 22-23 x' split (cinv only) | 8-11 P2^T
@@ -50,18 +56,25 @@ namespace kq {
 // Nonzero when a bounded wait gave up; each site ORs its own bit.
 __device__ unsigned int g_device_error = 0;
 
+// The word's device address, looked up once per device.  Only a successful
+// lookup is kept: a failed one (e.g. made during a stream capture) is returned
+// to the caller and tried again by the next launch.
 cudaError_t device_error_word(int device, unsigned int **word) {
-    static std::once_flag once[64];
+    static std::mutex mu;
     static unsigned int *addr[64];
-    static cudaError_t err[64];
     if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
-    std::call_once(once[device], [&] {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[device]) {
         void *p = nullptr;
-        err[device] = cudaGetSymbolAddress(&p, g_device_error);
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_device_error);
+        if (e != cudaSuccess) {
+            *word = nullptr;
+            return e;
+        }
         addr[device] = static_cast<unsigned int *>(p);
-    });
+    }
     *word = addr[device];
-    return err[device];
+    return cudaSuccess;
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, unsigned int *code) {
@@ -208,17 +221,15 @@ __device__ __forceinline__ void split_pair_neg(uint32_t v0, uint32_t v1, uint32_
 // adding 1.5 * 2^23 leaves the rounded integer in the low mantissa bits (bit
 // pattern 0x4B400000 + k).  The offset is removed by an integer multiply-add
 // with `one` (== 1, loaded at run time), which runs beside the floating-point
-// work instead of on the logic pipe.  (A packed fp32x2 form needs register
-// pairs the TMEM loads do not provide, and costs more instructions.)
+// work instead of on the logic pipe.  (A packed fp32x2 multiply-add for two
+// values at once needs register pairs the TMEM loads do not provide: it measured
+// 1-4 % slower over the whole kernel.)
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;  // 1.5 * 2^23
-// Two values at once: one packed fp32x2 multiply-add, then the two offsets removed.
-__device__ __forceinline__ void round_code2(uint32_t y0, uint32_t y1, uint64_t inv2, int one, int &k0, int &k1) {
-    const uint64_t y = uint64_t(y0) | (uint64_t(y1) << 32);
-    const uint64_t magic = (uint64_t(kRoundMagicBits) << 32) | kRoundMagicBits;
-    uint64_t b;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(b) : "l"(y), "l"(inv2), "l"(magic));
-    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k0) : "r"(uint32_t(b)), "r"(one), "r"(-int(kRoundMagicBits)));
-    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k1) : "r"(uint32_t(b >> 32)), "r"(one), "r"(-int(kRoundMagicBits)));
+__device__ __forceinline__ int round_code(uint32_t ybits, float inv, int one) {
+    const uint32_t b = __float_as_uint(fmaf(__uint_as_float(ybits), inv, 12582912.0f));
+    int k;
+    asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(k) : "r"(b), "r"(one), "r"(-int(kRoundMagicBits)));
+    return k;
 }
 
 
@@ -841,7 +852,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // exact quotients by a few ulps, far inside the rounding-boundary window
             const float s = alpha * m * (1.0f / 7.0f);
             const float inv = s > 0.0f ? fminf(__fdividef(1.0f, s), 3.0e38f) : 0.0f;
-            const uint64_t inv2 = (uint64_t(__float_as_uint(inv)) << 32) | __float_as_uint(inv);
             unsigned char *stg = smem + C::OFF_STG + (2 * ew + buf) * C::STG;
             // this thread's two bytes of every row: columns 4 g8 .. 4 g8 + 3 of the warp's 32.
             // It writes rows row0 + 16 c + 8 rep + 2 qq + d, whose swizzle term of
@@ -874,10 +884,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     // rows i0 + d, i0 = 16 c0 + 8 rep + 2 qq: registers 4 rep + d hold the even
                     // column, 4 rep + 2 + d the odd one, of half 0 (ra) and half 1 (rb)
                     int ka[4], kb[4];
-                    round_code2(ra[4 * rep], ra[4 * rep + 1], inv2, one, ka[0], ka[1]);
-                    round_code2(ra[4 * rep + 2], ra[4 * rep + 3], inv2, one, ka[2], ka[3]);
-                    round_code2(rb[4 * rep], rb[4 * rep + 1], inv2, one, kb[0], kb[1]);
-                    round_code2(rb[4 * rep + 2], rb[4 * rep + 3], inv2, one, kb[2], kb[3]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        ka[e] = round_code(ra[4 * rep + e], inv, one);
+                        kb[e] = round_code(rb[4 * rep + e], inv, one);
+                    }
 #pragma unroll
                     for (int d = 0; d < 2; ++d) {
                         // row i0 + d: columns 4 g8 + (0, 1) from half 0, + (2, 3) from half 1;
