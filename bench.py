@@ -62,7 +62,8 @@ def parse():
                          "of packed codes that consumes it (M = N = K = 8192); two_stage: the path for "
                          "factors above 128 (--two-stage-config); headwise: the per-head key/value "
                          "transform + INT4 (8192 tokens x 32 heads x 128)")
-    ap.add_argument("--config", choices=["hidden8192", "llama7b_hidden", "mlp14336", "mlp14336_cinv", "sweep4096"],
+    ap.add_argument("--config", choices=["hidden8192", "llama7b_hidden", "mlp14336", "mlp14336_cinv", "hidden5120",
+                                         "sweep4096"],
                     default=WORKLOAD,
                     help="configuration of the transform workload (both arms); the default is the headline one")
     ap.add_argument("--two-stage-config", choices=["square65536", "ffn28672"], default="square65536")

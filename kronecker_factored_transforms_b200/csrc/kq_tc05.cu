@@ -136,7 +136,12 @@ __host__ __device__ constexpr int imax(int a, int b) { return a > b ? a : b; }
 
 template <int N1, int N2, bool SCALED>
 struct Cfg {
-    static constexpr int H = 128 / N2;               // tokens stacked in the TMEM lanes
+    // The tile layout works on N2P = 64 or 128 columns per token; n2 = 48 (80, 96,
+    // 112) is padded to 64 (128): the x boxes read zeros past n2, the padded rows
+    // and columns of P2^T are zero, and no code is stored for them.
+    static constexpr int N2P = N2 <= 64 ? 64 : 128;
+    static constexpr bool PADDED = N2 != N2P;
+    static constexpr int H = 128 / N2P;              // tokens stacked in the TMEM lanes
     // Stage 1 runs on batches of GB groups so that its MMAs are N = GB * n1 wide
     // (up to 128).
     static constexpr int GB = N1 <= 64 ? imin(8, 128 / N1) : 1;
@@ -154,11 +159,13 @@ struct Cfg {
     static constexpr int TMEM_USED = A1COLS + NB1 * R1W + NB2 * N1P;
     static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
     static constexpr int RB = N2 / 2;                // bytes of one output row (codes)
-    static constexpr int STG = H * N1 * RB;          // staging bytes per group (a multiple of 1024)
+    // staging bytes per group: a multiple of 1024 (the swizzled TMA-store tile) or,
+    // padded, of 128 (rows in plain order, written out by one bulk copy)
+    static constexpr int STG = H * N1 * RB;
     static constexpr int OFF_B2 = 0;
     static constexpr int OFF_A1 = align_up(OFF_B2 + NCH2 * N1 * 128, 1024);
     static constexpr int OFF_STG = OFF_A1 + (A1_TMEM ? 0 : 32768);  // 2 epilogues x 2 staging buffers
-    static constexpr int OFF_RAW = OFF_STG + 4 * STG;
+    static constexpr int OFF_RAW = align_up(OFF_STG + 4 * STG, 1024);
     static constexpr int BUDGET = 222 * 1024 - OFF_RAW - 2048;
     static constexpr int SC = (SCALED && BUDGET >= 10 * XTILE) ? 4 : 2;  // lo-half tile stages (cinv)
     static constexpr int SX = imax(2, imin(8, (BUDGET - (SCALED ? SC * XTILE : 0)) / XTILE));  // raw x stages
@@ -184,12 +191,13 @@ struct Cfg {
     static constexpr int D2FULL = D1EMPTY + NB1, D2EMPTY = D2FULL + NB2, TEARDOWN = D2EMPTY + NB2;
     static constexpr int FACT = TEARDOWN + 1;  // P1 and P2 landed in the scratch
     static_assert(SX > NSCR_RAW && NSCR - NSCR_RAW <= (SCALED ? SC : 0) , "at least one x stage besides the factor scratch");
-    static_assert(N2 == 64 || N2 == 128, "stage 1 needs K = H * n2 = 128");
+    static_assert(N2 % 16 == 0 && N2 >= 48 && N2 <= 128, "stage 1 needs K = H * n2 (padded) = 128");
     static_assert(N1 % 16 == 0 && N1 >= 16 && N1 <= 128, "n1 must be a multiple of 16 in [16, 128]");
     static_assert(NS1 % 16 == 0 && NS1 <= 128, "stage-1 MMA width");
     static_assert(NB1 >= 2, "stage-1 regions");
     static_assert(TMEM_USED <= 512, "TMEM budget");
-    static_assert(STG % 1024 == 0 && OFF_STG % 1024 == 0 && OFF_RAW % 1024 == 0, "swizzle alignment");
+    static_assert((PADDED ? STG % 128 : STG % 1024) == 0 && OFF_STG % 1024 == 0 && OFF_RAW % 1024 == 0,
+                  "swizzle and bulk-copy alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
     __host__ __device__ static constexpr uint32_t R1(int b) { return uint32_t(A1COLS + b * R1W); }
     __host__ __device__ static constexpr uint32_t R2(int b) { return uint32_t(A1COLS + NB1 * R1W + b * N1P); }
@@ -238,9 +246,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     kq_tc05_fused_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
                          const uint16_t *__restrict__ P1,
                          const uint16_t *__restrict__ P2, const float *__restrict__ cinv, float alpha,
-                         float *__restrict__ scale_out, int64_t T) {
+                         uint8_t *__restrict__ q_out, float *__restrict__ scale_out, int64_t T) {
     using C = Cfg<N1, N2, SCALED>;
-    static_assert(staging_addresses_match<N1, N2>(), "epilogue staging addresses");
+    constexpr int N2P = C::N2P;
+    static_assert(C::PADDED || staging_addresses_match<N1, N2>(), "epilogue staging addresses");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
@@ -357,8 +366,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int u = 0; u < PER; ++u) {
                 const int c = st + u * kSetupThreads;
                 const int l = c % 128, k0 = 8 * (c / 128);
-                const int h = l / N2, j = lane_column(l % N2), hk = k0 / N2, b0 = k0 % N2;
-                const bool on = c < PIECES && h == hk;
+                const int h = l / N2P, j = lane_column(l % N2P), hk = k0 / N2P, b0 = k0 % N2P;
+                // (eight K values never straddle n2: both are multiples of 8)
+                const bool on = c < PIECES && h == hk && j < N2 && b0 < N2;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const uint32_t lo = on ? P2s[(b0 + 2 * e) * N2 + j] : 0u;
@@ -389,7 +399,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int k = 32 * (kc0 + kq) + 2 * e;
-                    w[kq][e] = uint32_t(a1_value<N2>(P2s, l, k)) | (uint32_t(a1_value<N2>(P2s, l, k + 1)) << 16);
+                    w[kq][e] = uint32_t(a1_value<N2, N2P>(P2s, l, k)) |
+                               (uint32_t(a1_value<N2, N2P>(P2s, l, k + 1)) << 16);
                 }
 #pragma unroll
             for (int kq = 0; kq < 2; ++kq) tmem_st_32x32b_x16(taddr + 16 * (kc0 + kq), w[kq]);
@@ -437,8 +448,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
                         const int64_t g = g0 + gp;
-                        const int xc = (N2 == 128) ? 64 * c : 0;
-                        const int64_t row = (N2 == 128) ? g * N1 : (2 * g + c) * N1;
+                        const int xc = (N2P == 128) ? 64 * c : 0;  // columns past n2 read as zero
+                        const int64_t row = (N2P == 128) ? g * N1 : (2 * g + c) * N1;
                         tma_load_2d(dst + c * C::CHUNK + gp * (N1 * 128), &tmap_x, xc, int(row),
                                     bar(C::FULL + rx.idx));
                     }
@@ -576,14 +587,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // MMA's negate-B bit; hi + lo is x cinv to about 2^-14 relative.
             const int t = 32 * xsplit_index(warp) + lane;  // 0 .. kXThreads - 1
             constexpr int UPT = 16 * N1 / kXThreads;       // units per thread per token
-            constexpr int UR = N1 == 96 ? 3 : 4, UG = UPT - UR;  // register units, cached units
+            constexpr int UR = (N1 == 96 || (C::PADDED && N1 == 112)) ? 3 : 4, UG = UPT - UR;  // register units, cached units
             static_assert(C::GB == 1 && UG >= 1 && UG <= 5, "one group per batch for n1 > 64");
             // unit e = t + kXThreads u: row r of chunk c, 16-byte column up of the
             // swizzled tile, i.e. channels r n2 + b0 .. + 7
+            // (-1 for a unit of the zero padding past n2)
             auto chan0 = [&](int u) {
                 const int e = t + kXThreads * u;
                 const int c = e / (8 * N1), rem = e % (8 * N1), r = rem >> 3, up = rem & 7;
-                return r * N2 + (N2 == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
+                const int b0 = (N2P == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
+                return (!C::PADDED || b0 < N2) ? r * N2 + b0 : -1;
+            };
+            auto load_c8 = [&](int ch, float4 &a, float4 &b) {
+                if (!C::PADDED || ch >= 0) {
+                    a = __ldg(reinterpret_cast<const float4 *>(cinv + ch));
+                    b = __ldg(reinterpret_cast<const float4 *>(cinv + ch + 4));
+                } else {
+                    a = b = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                }
             };
             auto tile_off = [&](int u) {
                 const int e = t + kXThreads * u;
@@ -593,10 +614,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             {
                 float4 ca[UR], cb[UR];  // every load first
 #pragma unroll
-                for (int u = 0; u < UR; ++u) {
-                    ca[u] = __ldg(reinterpret_cast<const float4 *>(cinv + chan0(u)));
-                    cb[u] = __ldg(reinterpret_cast<const float4 *>(cinv + chan0(u) + 4));
-                }
+                for (int u = 0; u < UR; ++u) load_c8(chan0(u), ca[u], cb[u]);
 #pragma unroll
                 for (int u = 0; u < UR; ++u) {
                     const float cv[8] = {ca[u].x, ca[u].y, ca[u].z, ca[u].w, cb[u].x, cb[u].y, cb[u].z, cb[u].w};
@@ -623,10 +641,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 constexpr int PF = UG < 2 ? UG : 2;
                 float4 ga[UG], gb[UG];
 #pragma unroll
-                for (int g = 0; g < PF; ++g) {
-                    ga[g] = __ldg(reinterpret_cast<const float4 *>(cinv + chan0(UR + g)));
-                    gb[g] = __ldg(reinterpret_cast<const float4 *>(cinv + chan0(UR + g) + 4));
-                }
+                for (int g = 0; g < PF; ++g) load_c8(chan0(UR + g), ga[g], gb[g]);
 #pragma unroll
                 for (int u = 0; u < UR; ++u) {
                     const int off = tile_off(u);
@@ -644,10 +659,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
 #pragma unroll
                 for (int g = 0; g < UG; ++g) {
-                    if (g + PF < UG) {  // keep PF loads in flight
-                        ga[g + PF] = __ldg(reinterpret_cast<const float4 *>(cinv + chan0(UR + g + PF)));
-                        gb[g + PF] = __ldg(reinterpret_cast<const float4 *>(cinv + chan0(UR + g + PF) + 4));
-                    }
+                    if (g + PF < UG) load_c8(chan0(UR + g + PF), ga[g + PF], gb[g + PF]);  // keep PF loads in flight
                     const int off = tile_off(UR + g);
                     const uint4 in = *reinterpret_cast<const uint4 *>(raw + off);
                     const uint32_t w[4] = {in.x, in.y, in.z, in.w};
@@ -681,9 +693,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int u = 0; u < UPT; ++u) {
                 const int e = t + kXThreads * u;
                 const int c = e / (8 * N1), rem = e % (8 * N1), r = rem >> 3, up = rem & 7;
-                const int b0 = (N2 == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
-                ca[u] = __ldg(reinterpret_cast<const float4 *>(cinv + r * N2 + b0));
-                cb[u] = __ldg(reinterpret_cast<const float4 *>(cinv + r * N2 + b0 + 4));
+                const int b0 = (N2P == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
+                if (!C::PADDED || b0 < N2) {
+                    ca[u] = __ldg(reinterpret_cast<const float4 *>(cinv + r * N2 + b0));
+                    cb[u] = __ldg(reinterpret_cast<const float4 *>(cinv + r * N2 + b0 + 4));
+                } else {  // zero padding past n2
+                    ca[u] = cb[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                }
             }
 #pragma unroll
             for (int u = 0; u < UPT; ++u) {
@@ -772,7 +788,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int q = warp & 3;
         const int et = tid - 384 - 128 * ew;
         const uint32_t nbar = 1u + uint32_t(ew);
-        const int tok_h = (32 * q) / N2;
+        const int tok_h = (32 * q) / N2P;
         const int g8 = lane >> 2, qq = lane & 3;
         float *red = s_red + 8 * ew;
         const int one = *reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
@@ -780,11 +796,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t ng = uint32_t(nb) * C::GB;
         const uint32_t stg0 = sbase + C::OFF_STG + 2 * ew * C::STG;
         // One thread per warpgroup writes a finished staging tile to HBM with a
-        // TMA store; the tensor map clips rows past the last token.
+        // TMA store (the tensor map clips rows past the last token) or, for a padded
+        // n2, whose code rows are not a multiple of 16 bytes, with one bulk copy of
+        // the group's valid tokens (contiguous in q_out).
         const bool storer = et == 0;
         auto store_group = [&](int64_t gprev, int sb) {
             if (storer) {
-                tma_store_2d(&tmap_q, 0, int(C::H * gprev * N1), stg0 + uint32_t(sb) * C::STG);
+                if constexpr (C::PADDED) {
+                    // the last batch of a CTA can end in groups past the last token
+                    // (G not a multiple of GB): nothing of theirs is stored
+                    const int64_t tok0 = C::H * gprev, ntok = T - tok0 < C::H ? T - tok0 : C::H;
+                    if (ntok > 0)
+                        bulk_store(q_out + tok0 * (N1 * C::RB), stg0 + uint32_t(sb) * C::STG,
+                                   uint32_t(ntok * N1 * C::RB));
+                } else {
+                    tma_store_2d(&tmap_q, 0, int(C::H * gprev * N1), stg0 + uint32_t(sb) * C::STG);
+                }
                 bulk_commit();
             }
         };
@@ -847,7 +874,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             float m = 0.0f;
 #pragma unroll
             for (int w = 0; w < 4; ++w)
-                if ((32 * w) / N2 == tok_h) m = fmaxf(m, red[4 * buf + w]);
+                if ((32 * w) / N2P == tok_h) m = fmaxf(m, red[4 * buf + w]);
             // s = alpha * max / 7 to within an ulp; codes use y * (1/s): both differ from the
             // exact quotients by a few ulps, far inside the rounding-boundary window
             const float s = alpha * m * (1.0f / 7.0f);
@@ -858,9 +885,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // stg_offset is the same for all of them: qq (64-byte rows; row0 is a
             // multiple of 16) or qq >> 1 (32-byte rows).  So every store is one base
             // address plus a constant.
-            const int row0 = tok_h * N1, bcol = ((32 * q) % N2) / 2 + 2 * g8;
-            const int swz_t = N2 == 128 ? qq : (qq >> 1);
-            unsigned char *tbase = stg + (row0 + 2 * qq) * C::RB + ((((bcol >> 4) ^ swz_t) << 4) | (bcol & 15));
+            const int row0 = tok_h * N1, bcol = ((32 * q) % N2P) / 2 + 2 * g8;
+            // padded n2: rows in plain order, and no store for the columns past n2
+            const bool keep = !C::PADDED || bcol < C::RB;
+            const int swz_t = N2P == 128 ? qq : (qq >> 1);
+            unsigned char *tbase = stg + (row0 + 2 * qq) * C::RB +
+                                   (C::PADDED ? bcol : ((((bcol >> 4) ^ swz_t) << 4) | (bcol & 15)));
             const uint32_t t0 = tmem + (uint32_t(32 * q) << 16) + C::R2(int(b));
             constexpr int CB = N1 % 32 == 0 ? 2 : 1;  // 16-column chunks per load
 #pragma unroll
@@ -895,13 +925,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         // byte = even column in the low nibble, odd in the high one
                         const uint32_t wb = pack_s4x2(kb[2 + d], kb[d], 0u);
                         const uint32_t w = pack_s4x2(ka[2 + d], ka[d], wb);
-                        *reinterpret_cast<uint16_t *>(tbase + (16 * c0 + 8 * rep + d) * C::RB) = uint16_t(w);
+                        if (keep) *reinterpret_cast<uint16_t *>(tbase + (16 * c0 + 8 * rep + d) * C::RB) = uint16_t(w);
                     }
                 }
             }
             fence_proxy_async_smem();  // staging writes visible to the TMA store
             const int64_t tok0 = C::H * g;
-            if (lane == 0 && (32 * q) % N2 == 0 && tok0 + tok_h < T) scale_out[tok0 + tok_h] = s;
+            if (lane == 0 && (32 * q) % N2P == 0 && tok0 + tok_h < T) scale_out[tok0 + tok_h] = s;
             g_prev = g;
         }
         // the last group's rows: everyone has written them once all pass this barrier
@@ -959,14 +989,17 @@ cudaError_t launch_inst(const LaunchArgs &a) {
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     // codes: rows of n2/2 bytes, one box = one group's H * n1 rows, swizzled like the staging tile
-    CUtensorMap tmap_q;
-    const cuuint64_t qdims[2] = {cuuint64_t(C::RB), cuuint64_t(a.T) * N1};
-    const cuuint64_t qstrides[1] = {cuuint64_t(C::RB)};
-    const cuuint32_t qbox[2] = {cuuint32_t(C::RB), cuuint32_t(C::H * N1)};
-    r = encode(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.q_out, qdims, qstrides, qbox, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, N2 == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B,
-               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    // (a padded n2 stores its codes by bulk copies instead; the map is then unused)
+    CUtensorMap tmap_q = tmap;
+    if constexpr (!C::PADDED) {
+        const cuuint64_t qdims[2] = {cuuint64_t(C::RB), cuuint64_t(a.T) * N1};
+        const cuuint64_t qstrides[1] = {cuuint64_t(C::RB)};
+        const cuuint32_t qbox[2] = {cuuint32_t(C::RB), cuuint32_t(C::H * N1)};
+        r = encode(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.q_out, qdims, qstrides, qbox, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, N2 == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
     const int64_t G = (a.T + C::H - 1) / C::H;
     const int64_t NBt = (G + C::GB - 1) / C::GB;
     const int64_t grid = NBt < a.num_sms ? NBt : a.num_sms;
@@ -974,7 +1007,7 @@ cudaError_t launch_inst(const LaunchArgs &a) {
     // the stream is another launch of this kernel, this grid's launch and set-up
     // overlap that grid's last CTAs (see griddep_launch_dependents / griddep_wait).
     return launch_overlapped(kern, unsigned(grid), kTcThreads, C::SMEM, a.stream, tmap, tmap_q, a.P1, a.P2, a.cinv,
-                             a.alpha, a.scale_out, a.T);
+                             a.alpha, a.q_out, a.scale_out, a.T);
 }
 
 template <int N2, bool SCALED>
@@ -1013,15 +1046,22 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 bool tc05_supports(int n1, int n2, bool scaled) {
     (void)scaled;
-    if (n2 != 64 && n2 != 128) return false;
+    if (n2 < 48 || n2 > 128 || n2 % 16 != 0) return false;  // n2 = 48, 80, 96, 112 run padded
     return n1 >= 16 && n1 <= 128 && n1 % 16 == 0;
 }
 
 cudaError_t launch_tc05(const LaunchArgs &a) {
     if (a.T * int64_t(a.n1) >= (int64_t(1) << 31)) return launch_warp_mma(a);  // TMA row coordinate range
     const bool scaled = a.cinv != nullptr;
-    if (a.n2 == 128) return scaled ? dispatch_n1<128, true>(a) : dispatch_n1<128, false>(a);
-    return scaled ? dispatch_n1<64, true>(a) : dispatch_n1<64, false>(a);
+    switch (a.n2) {
+    case 48: return scaled ? dispatch_n1<48, true>(a) : dispatch_n1<48, false>(a);
+    case 64: return scaled ? dispatch_n1<64, true>(a) : dispatch_n1<64, false>(a);
+    case 80: return scaled ? dispatch_n1<80, true>(a) : dispatch_n1<80, false>(a);
+    case 96: return scaled ? dispatch_n1<96, true>(a) : dispatch_n1<96, false>(a);
+    case 112: return scaled ? dispatch_n1<112, true>(a) : dispatch_n1<112, false>(a);
+    case 128: return scaled ? dispatch_n1<128, true>(a) : dispatch_n1<128, false>(a);
+    default: return cudaErrorNotSupported;
+    }
 }
 
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream) {

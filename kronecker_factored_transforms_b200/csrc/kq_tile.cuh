@@ -70,11 +70,12 @@ static_assert(lane_maps_invert(), "lane_of_column inverts lane_column");
 
 // Row l of A1 = block-diag over the stacked tokens of P2^T, rows permuted:
 // A1[l][k] = P2[b][lane_column(m)] for l = (h, m), k = (h, b); zero off the
-// diagonal blocks.
-template <int N2>
+// diagonal blocks.  Tokens take N2P >= n2 lanes and K values each; rows and
+// columns past n2 (a padded n2) are zero.
+template <int N2, int N2P = N2>
 __device__ __forceinline__ uint16_t a1_value(const uint16_t *__restrict__ P2, int l, int k) {
-    const int h = l / N2, m = l % N2, hk = k / N2, b = k % N2;
-    return (h == hk) ? P2[b * N2 + lane_column(m)] : uint16_t(0);
+    const int h = l / N2P, m = l % N2P, hk = k / N2P, b = k % N2P, j = lane_column(m);
+    return (h == hk && b < N2 && j < N2) ? P2[b * N2 + j] : uint16_t(0);
 }
 
 }  // namespace tile

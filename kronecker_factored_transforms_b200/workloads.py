@@ -122,6 +122,11 @@ CONFIGS = {
     "mlp14336_cinv": dict(T=4096, n1=112, n2=128, seed=7, alpha=0.9, factors="orthogonal",
                           x_kind="relu_gated", outliers=("frac", 0.005, 40.0), pivot=None,
                           scaled=True),
+    # n=5120 (64x80), the hidden size of a 13B-class model: an n2 outside
+    # {64, 128}; the hidden8192 recipe otherwise (Student-t, c ~ logU[0.5, 2],
+    # near-identity factors, alpha = 0.85); seed 8.
+    "hidden5120": dict(T=4096, n1=64, n2=80, seed=8, alpha=0.85, factors="near_identity",
+                       x_kind="student_t", outliers=None, pivot=None, scaled=True),
     # n=4096 (64x64) at T in SWEEP_T; N(0,1) + 1% x30; orthogonal;
     # alpha = 0.9; seed 4.
     "sweep4096": dict(T=1024, n1=64, n2=64, seed=4, alpha=0.9, factors="orthogonal",

@@ -59,6 +59,24 @@ def test_kernel_name_for_shapes(kq):
     assert kq.kq_kernel_name(16, 144, False) == "unsupported"
 
 
+def test_kernel_selection_rules(kq):
+    """The dispatch rule, host side only (no GPU: kq_kernel_for assumes 148 SMs)."""
+    tc, pair, warp = "kq_tc05_fused_kernel", "kq_fused_kernel", "kq_warp_mma_kernel"
+    for n2 in (48, 64, 80, 96, 112, 128):  # n2 padded to 64 or 128 columns on the tensor cores
+        assert kq.kq_kernel_name(112, n2, True) == tc
+    for n2 in (16, 32):
+        assert kq.kq_kernel_name(64, n2, False) == warp
+    assert kq.kq_kernel_for(2048, 64, 64, False, 0.88) == pair      # short launch at n1 = 64
+    assert kq.kq_kernel_for(148 * 24, 64, 128, True, 0.85) == pair  # 24 groups per SM
+    assert kq.kq_kernel_for(148 * 24 + 1, 64, 128, True, 0.85) == tc
+    assert kq.kq_kernel_for(148 * 48, 64, 64, False, 0.9) == pair   # two tokens per group at n2 = 64
+    assert kq.kq_kernel_for(148 * 48 + 2, 64, 64, False, 0.9) == tc
+    assert kq.kq_kernel_for(16, 64, 80, True, 0.85) == tc           # the pair kernel has n2 in {64, 128} only
+    assert kq.kq_kernel_for(16, 112, 128, False, 0.9) == tc
+    assert kq.kq_kernel_for(16, 64, 64, False, 2.0 ** -20) == warp  # alpha below 2^-19
+    assert kq.kq_kernel_for(16, 24, 64, False, 0.9) == "unsupported"
+
+
 # Fake, never-dereferenced device addresses (validation rejects every call below).
 X, P1, P2, CI, Q, S, Y = 0x10000000, 0x20000000, 0x20010000, 0x20020000, 0x30000000, 0x40000000, 0x50000000
 

@@ -91,7 +91,7 @@ def assert_quant_parity(x, P1, P2, cinv, alpha, n1, n2, q_gpu, s_gpu, chunk=1024
 # ---------------------------------------------------------------------------
 # The five configurations at full size.
 
-@pytest.mark.parametrize("name", ["tiny", "llama7b_hidden", "hidden8192", "mlp14336", "mlp14336_cinv"])
+@pytest.mark.parametrize("name", ["tiny", "llama7b_hidden", "hidden8192", "mlp14336", "mlp14336_cinv", "hidden5120"])
 def test_config_full_size(kq, name):
     w = make_workload(name)
     q, s = run_quant(kq, w.x, w.P1, w.P2, w.cinv, w.alpha, w.T, w.n1, w.n2)
@@ -111,7 +111,7 @@ def test_sweep(kq, T):
         assert_quant_parity(w.x[rows], w.P1, w.P2, None, w.alpha, 64, 64, q[rows], s[rows])
 
 
-@pytest.mark.parametrize("name", ["tiny", "llama7b_hidden", "hidden8192", "mlp14336", "mlp14336_cinv"])
+@pytest.mark.parametrize("name", ["tiny", "llama7b_hidden", "hidden8192", "mlp14336", "mlp14336_cinv", "hidden5120"])
 def test_transform_check_entry(kq, name):
     w = make_workload(name, rows=512 if name != "tiny" else None)
     T = w.x.shape[0]
@@ -127,7 +127,9 @@ def test_transform_check_entry(kq, name):
 # Shapes, ragged sizes and degenerate inputs.
 
 SHAPES = [(16, 16), (16, 128), (128, 16), (32, 48), (48, 32), (64, 64), (64, 128), (112, 128),
-          (128, 128), (80, 96), (80, 64), (96, 128), (112, 64), (128, 64)]
+          (128, 128), (80, 96), (80, 64), (96, 128), (112, 64), (128, 64),
+          # n2 padded to 64 or 128 columns on the tensor cores
+          (64, 80), (16, 48), (128, 48), (112, 112), (96, 80), (128, 112), (48, 96)]
 
 
 @pytest.mark.parametrize("n1,n2", SHAPES)
@@ -252,9 +254,13 @@ def test_fast_kernel_is_selected_for_the_configs(kq):
     assert kq.kq_kernel_for(2048, 64, 64, False, 0.88) == "kq_fused_kernel"        # llama7b_hidden
     assert kq.kq_kernel_for(1, 64, 128, True, 0.85) == "kq_fused_kernel"
     assert kq.kq_kernel_for(4096, 112, 128, False, 0.9) == "kq_tc05_fused_kernel"  # mlp14336
-    for n1 in (80, 96, 112, 128):  # cinv with n1 > 64 (the factor scratch may take the lo stages)
-        for n2 in (64, 128):
-            assert kq.kq_kernel_name(n1, n2, True) == "kq_tc05_fused_kernel", (n1, n2)
+    for n1 in (16, 48, 64, 80, 96, 112, 128):  # cinv with n1 > 64; n2 padded to 64 or 128
+        for n2 in (48, 64, 80, 96, 112, 128):
+            for scaled in (False, True):
+                assert kq.kq_kernel_name(n1, n2, scaled) == "kq_tc05_fused_kernel", (n1, n2, scaled)
+    assert kq.kq_kernel_for(4096, 64, 80, True, 0.85) == "kq_tc05_fused_kernel"     # hidden5120
+    for n2 in (16, 32):
+        assert kq.kq_kernel_name(64, n2, True) == "kq_warp_mma_kernel"
     assert kq.kq_kernel_for(64, 64, 64, False, 1e-7) == "kq_warp_mma_kernel"
     assert kq.kq_kernel_name(16, 16, False) == "kq_warp_mma_kernel"
 

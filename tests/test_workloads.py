@@ -21,7 +21,7 @@ def test_bf16_cast_is_round_to_nearest_even():
 
 
 @pytest.mark.parametrize("name", ["tiny", "llama7b_hidden", "hidden8192", "mlp14336", "mlp14336_cinv",
-                                  "sweep4096", "ffn28672", "square65536"])
+                                  "hidden5120", "sweep4096", "ffn28672", "square65536"])
 def test_shapes_and_reproducibility(name):
     a = make_workload(name, rows=8)
     b = make_workload(name, rows=8)
