@@ -138,9 +138,15 @@ template <int N1, int N2, bool SCALED>
 struct Cfg {
     // The tile layout works on N2P = 64 or 128 columns per token; n2 = 48 (80, 96,
     // 112) is padded to 64 (128): the x boxes read zeros past n2, the padded rows
-    // and columns of P2^T are zero, and no code is stored for them.
+    // and columns of P2^T are zero, and no code is stored for them.  (n2 = 16 and
+    // 32 would need two or four tokens side by side in one 128-byte row of a K
+    // chunk; a 128-byte-swizzled TMA box narrower than 128 bytes still takes 128
+    // bytes per row in shared memory, so one box cannot place them.)
     static constexpr int N2P = N2 <= 64 ? 64 : 128;
     static constexpr bool PADDED = N2 != N2P;
+    // codes staged in plain row order and stored by one bulk copy per group (rows
+    // of n2/2 bytes that are not 32 or 64: no swizzled tensor store for them)
+    static constexpr bool PLAIN = PADDED;
     static constexpr int H = 128 / N2P;              // tokens stacked in the TMEM lanes
     // Stage 1 runs on batches of GB groups so that its MMAs are N = GB * n1 wide
     // (up to 128).
@@ -160,7 +166,7 @@ struct Cfg {
     static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
     static constexpr int RB = N2 / 2;                // bytes of one output row (codes)
     // staging bytes per group: a multiple of 1024 (the swizzled TMA-store tile) or,
-    // padded, of 128 (rows in plain order, written out by one bulk copy)
+    // PLAIN, of 128 (rows in plain order, written out by one bulk copy)
     static constexpr int STG = H * N1 * RB;
     static constexpr int OFF_B2 = 0;
     static constexpr int OFF_A1 = align_up(OFF_B2 + NCH2 * N1 * 128, 1024);
@@ -196,7 +202,7 @@ struct Cfg {
     static_assert(NS1 % 16 == 0 && NS1 <= 128, "stage-1 MMA width");
     static_assert(NB1 >= 2, "stage-1 regions");
     static_assert(TMEM_USED <= 512, "TMEM budget");
-    static_assert((PADDED ? STG % 128 : STG % 1024) == 0 && OFF_STG % 1024 == 0 && OFF_RAW % 1024 == 0,
+    static_assert((PLAIN ? STG % 128 : STG % 1024) == 0 && OFF_STG % 1024 == 0 && OFF_RAW % 1024 == 0,
                   "swizzle and bulk-copy alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
     __host__ __device__ static constexpr uint32_t R1(int b) { return uint32_t(A1COLS + b * R1W); }
@@ -249,7 +255,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                          uint8_t *__restrict__ q_out, float *__restrict__ scale_out, int64_t T) {
     using C = Cfg<N1, N2, SCALED>;
     constexpr int N2P = C::N2P;
-    static_assert(C::PADDED || staging_addresses_match<N1, N2>(), "epilogue staging addresses");
+    static_assert(C::PLAIN || staging_addresses_match<N1, N2>(), "epilogue staging addresses");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
@@ -576,7 +582,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (xsplit_index(warp) >= 0) {
         // ---------------- x' = x * cinv -> hi / lo bf16 tiles ----------------
         if constexpr (SCALED && N1 > 64) {
-            // n1 > 64: 5 to 8 units per thread.  The first UR units keep their cinv in
+            // n1 > 64: 5 to 8 units per thread.  The first UR (3 or 4) units keep their cinv in
             // registers as two bf16 values, cinv = ch + cl (RN(cinv) and RN of the
             // rest): hi = RN(x ch), -lo = RN(-x cl + RN(-x ch + hi)), three packed bf16
             // operations per pair.  The other units read their cinv through the
@@ -587,7 +593,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // MMA's negate-B bit; hi + lo is x cinv to about 2^-14 relative.
             const int t = 32 * xsplit_index(warp) + lane;  // 0 .. kXThreads - 1
             constexpr int UPT = 16 * N1 / kXThreads;       // units per thread per token
-            constexpr int UR = (N1 == 96 || (C::PADDED && N1 == 112)) ? 3 : 4, UG = UPT - UR;  // register units, cached units
+            // register units, cached units (three register units where four leave the
+            // kernel short of registers: n1 = 96, and n1 >= 112 with a padded n2 or stacked tokens)
+            constexpr int UR = (N1 == 96 || (C::PADDED && N1 == 112) || (C::H > 1 && N1 >= 112)) ? 3 : 4;
+            constexpr int UG = UPT - UR;
             static_assert(C::GB == 1 && UG >= 1 && UG <= 5, "one group per batch for n1 > 64");
             // unit e = t + kXThreads u: row r of chunk c, 16-byte column up of the
             // swizzled tile, i.e. channels r n2 + b0 .. + 7
@@ -595,7 +604,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             auto chan0 = [&](int u) {
                 const int e = t + kXThreads * u;
                 const int c = e / (8 * N1), rem = e % (8 * N1), r = rem >> 3, up = rem & 7;
-                const int b0 = (N2P == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
+                const int b0 = (N2P == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));  // column within a token
                 return (!C::PADDED || b0 < N2) ? r * N2 + b0 : -1;
             };
             auto load_c8 = [&](int ch, float4 &a, float4 &b) {
@@ -693,7 +702,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int u = 0; u < UPT; ++u) {
                 const int e = t + kXThreads * u;
                 const int c = e / (8 * N1), rem = e % (8 * N1), r = rem >> 3, up = rem & 7;
-                const int b0 = (N2P == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));
+                const int b0 = (N2P == 128 ? 64 * c : 0) + 8 * (up ^ (r & 7));  // column within a token
                 if (!C::PADDED || b0 < N2) {
                     ca[u] = __ldg(reinterpret_cast<const float4 *>(cinv + r * N2 + b0));
                     cb[u] = __ldg(reinterpret_cast<const float4 *>(cinv + r * N2 + b0 + 4));
@@ -793,6 +802,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float *red = s_red + 8 * ew;
         const int one = *reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
         constexpr int NK = N1 / 16;
+        // 32-column TMEM loads; 16-column ones where the split warps hold cinv in
+        // registers (n1 > 64), which leaves fewer registers to this role
+        constexpr bool WIDE = N1 % 32 == 0 && !(SCALED && N1 > 64);
         const uint32_t ng = uint32_t(nb) * C::GB;
         const uint32_t stg0 = sbase + C::OFF_STG + 2 * ew * C::STG;
         // One thread per warpgroup writes a finished staging tile to HBM with a
@@ -802,7 +814,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool storer = et == 0;
         auto store_group = [&](int64_t gprev, int sb) {
             if (storer) {
-                if constexpr (C::PADDED) {
+                if constexpr (C::PLAIN) {
                     // the last batch of a CTA can end in groups past the last token
                     // (G not a multiple of GB): nothing of theirs is stored
                     const int64_t tok0 = C::H * gprev, ntok = T - tok0 < C::H ? T - tok0 : C::H;
@@ -832,7 +844,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             float mx4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             {
                 const uint32_t lane_off = uint32_t(32 * q) << 16;
-                if (N1 % 32 == 0) {
+                if (WIDE) {
 #pragma unroll
                     for (int k0 = 0; k0 < N1; k0 += 32) {
                         uint32_t v[32];
@@ -886,13 +898,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // multiple of 16) or qq >> 1 (32-byte rows).  So every store is one base
             // address plus a constant.
             const int row0 = tok_h * N1, bcol = ((32 * q) % N2P) / 2 + 2 * g8;
-            // padded n2: rows in plain order, and no store for the columns past n2
+            // plain staging: rows in order, and no store for the columns past n2
             const bool keep = !C::PADDED || bcol < C::RB;
             const int swz_t = N2P == 128 ? qq : (qq >> 1);
             unsigned char *tbase = stg + (row0 + 2 * qq) * C::RB +
-                                   (C::PADDED ? bcol : ((((bcol >> 4) ^ swz_t) << 4) | (bcol & 15)));
+                                   (C::PLAIN ? bcol : ((((bcol >> 4) ^ swz_t) << 4) | (bcol & 15)));
             const uint32_t t0 = tmem + (uint32_t(32 * q) << 16) + C::R2(int(b));
-            constexpr int CB = N1 % 32 == 0 ? 2 : 1;  // 16-column chunks per load
+            constexpr int CB = WIDE ? 2 : 1;  // 16-column chunks per load
 #pragma unroll
             for (int c0 = 0; c0 < NK; c0 += CB) {
                 // half 0 (lanes 32 q + [0, 16)) and half 1 (lanes 32 q + [16, 32))
@@ -980,18 +992,20 @@ cudaError_t launch_inst(const LaunchArgs &a) {
     PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
     if (!encode) return cudaErrorNotSupported;
     CUtensorMap tmap;
+    const cuuint32_t estr[2] = {1u, 1u};
+    // x as [T n1 rows][n2 columns]; one box = 64 columns (zeros past n2) by n1 rows,
+    // a full 128-byte swizzle row per tile row
     const cuuint64_t dims[2] = {cuuint64_t(N2), cuuint64_t(a.T) * N1};
     const cuuint64_t strides[1] = {cuuint64_t(N2) * 2};
     const cuuint32_t box[2] = {64u, cuuint32_t(N1)};
-    const cuuint32_t estr[2] = {1u, 1u};
     CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(a.x), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     // codes: rows of n2/2 bytes, one box = one group's H * n1 rows, swizzled like the staging tile
-    // (a padded n2 stores its codes by bulk copies instead; the map is then unused)
+    // (plain staging stores its codes by bulk copies instead; the map is then unused)
     CUtensorMap tmap_q = tmap;
-    if constexpr (!C::PADDED) {
+    if constexpr (!C::PLAIN) {
         const cuuint64_t qdims[2] = {cuuint64_t(C::RB), cuuint64_t(a.T) * N1};
         const cuuint64_t qstrides[1] = {cuuint64_t(C::RB)};
         const cuuint32_t qbox[2] = {cuuint32_t(C::RB), cuuint32_t(C::H * N1)};
