@@ -136,12 +136,13 @@ __host__ __device__ constexpr int imax(int a, int b) { return a > b ? a : b; }
 
 template <int N1, int N2, bool SCALED>
 struct Cfg {
-    // The tile layout works on N2P = 64 or 128 columns per token; n2 = 48 (80, 96,
-    // 112) is padded to 64 (128): the x boxes read zeros past n2, the padded rows
-    // and columns of P2^T are zero, and no code is stored for them.  (n2 = 16 and
-    // 32 would need two or four tokens side by side in one 128-byte row of a K
-    // chunk; a 128-byte-swizzled TMA box narrower than 128 bytes still takes 128
-    // bytes per row in shared memory, so one box cannot place them.)
+    // The tile layout works on N2P = 64 or 128 columns per token; n2 = 16, 32, 48
+    // (80, 96, 112) is padded to 64 (128): the x boxes read zeros past n2, the
+    // padded rows and columns of P2^T are zero, and no code is stored for them.
+    // (Stacking four or eight tokens of n2 = 32 or 16 in one 128-byte row of a K
+    // chunk would waste nothing, but a 128-byte-swizzled TMA box narrower than
+    // 128 bytes still takes 128 bytes per row in shared memory, so one box cannot
+    // place two tokens side by side.)
     static constexpr int N2P = N2 <= 64 ? 64 : 128;
     static constexpr bool PADDED = N2 != N2P;
     // codes staged in plain row order and stored by one bulk copy per group (rows
@@ -197,7 +198,7 @@ struct Cfg {
     static constexpr int D2FULL = D1EMPTY + NB1, D2EMPTY = D2FULL + NB2, TEARDOWN = D2EMPTY + NB2;
     static constexpr int FACT = TEARDOWN + 1;  // P1 and P2 landed in the scratch
     static_assert(SX > NSCR_RAW && NSCR - NSCR_RAW <= (SCALED ? SC : 0) , "at least one x stage besides the factor scratch");
-    static_assert(N2 % 16 == 0 && N2 >= 48 && N2 <= 128, "stage 1 needs K = H * n2 (padded) = 128");
+    static_assert(N2 % 16 == 0 && N2 >= 16 && N2 <= 128, "stage 1 needs K = H * n2 (padded) = 128");
     static_assert(N1 % 16 == 0 && N1 >= 16 && N1 <= 128, "n1 must be a multiple of 16 in [16, 128]");
     static_assert(NS1 % 16 == 0 && NS1 <= 128, "stage-1 MMA width");
     static_assert(NB1 >= 2, "stage-1 regions");
@@ -1060,7 +1061,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 bool tc05_supports(int n1, int n2, bool scaled) {
     (void)scaled;
-    if (n2 < 48 || n2 > 128 || n2 % 16 != 0) return false;  // n2 = 48, 80, 96, 112 run padded
+    if (n2 < 16 || n2 > 128 || n2 % 16 != 0) return false;  // n2 = 16, 32, 48, 80, 96, 112 run padded
     return n1 >= 16 && n1 <= 128 && n1 % 16 == 0;
 }
 
@@ -1068,6 +1069,8 @@ cudaError_t launch_tc05(const LaunchArgs &a) {
     if (a.T * int64_t(a.n1) >= (int64_t(1) << 31)) return launch_warp_mma(a);  // TMA row coordinate range
     const bool scaled = a.cinv != nullptr;
     switch (a.n2) {
+    case 16: return scaled ? dispatch_n1<16, true>(a) : dispatch_n1<16, false>(a);
+    case 32: return scaled ? dispatch_n1<32, true>(a) : dispatch_n1<32, false>(a);
     case 48: return scaled ? dispatch_n1<48, true>(a) : dispatch_n1<48, false>(a);
     case 64: return scaled ? dispatch_n1<64, true>(a) : dispatch_n1<64, false>(a);
     case 80: return scaled ? dispatch_n1<80, true>(a) : dispatch_n1<80, false>(a);

@@ -62,11 +62,9 @@ def test_kernel_name_for_shapes(kq):
 def test_kernel_selection_rules(kq):
     """The dispatch rule, host side only (no GPU: kq_kernel_for assumes 148 SMs)."""
     tc, pair, warp = "kq_tc05_fused_kernel", "kq_fused_kernel", "kq_warp_mma_kernel"
-    for n2 in (48, 64, 80, 96, 112, 128):  # n2 padded to 64 or 128 columns where needed
+    for n2 in (16, 32, 48, 64, 80, 96, 112, 128):  # n2 padded to 64 or 128 columns where needed
         assert kq.kq_kernel_name(112, n2, True) == tc
         assert kq.kq_kernel_name(16, n2, False) == tc
-    for n2 in (16, 32):
-        assert kq.kq_kernel_name(64, n2, False) == warp
     assert kq.kq_kernel_for(2048, 64, 64, False, 0.88) == pair      # short launch at n1 = 64
     assert kq.kq_kernel_for(148 * 24, 64, 128, True, 0.85) == pair  # 24 groups per SM
     assert kq.kq_kernel_for(148 * 24 + 1, 64, 128, True, 0.85) == tc

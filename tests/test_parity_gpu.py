@@ -130,7 +130,6 @@ SHAPES = [(16, 16), (16, 128), (128, 16), (32, 48), (48, 32), (64, 64), (64, 128
           (128, 128), (80, 96), (80, 64), (96, 128), (112, 64), (128, 64),
           # n2 padded to 64 or 128 columns on the tensor cores
           (64, 80), (16, 48), (128, 48), (112, 112), (96, 80), (128, 112), (48, 96),
-          # n2 = 16 and 32 (the warp-MMA kernel)
           (64, 32), (112, 16), (32, 32), (128, 32), (80, 16)]
 
 
@@ -257,13 +256,11 @@ def test_fast_kernel_is_selected_for_the_configs(kq):
     assert kq.kq_kernel_for(1, 64, 128, True, 0.85) == "kq_fused_kernel"
     assert kq.kq_kernel_for(4096, 112, 128, False, 0.9) == "kq_tc05_fused_kernel"  # mlp14336
     for n1 in (16, 48, 64, 80, 96, 112, 128):  # cinv with n1 > 64; n2 padded to 64 or 128
-        for n2 in (48, 64, 80, 96, 112, 128):
+        for n2 in (16, 32, 48, 64, 80, 96, 112, 128):
             for scaled in (False, True):
                 assert kq.kq_kernel_name(n1, n2, scaled) == "kq_tc05_fused_kernel", (n1, n2, scaled)
-        for n2 in (16, 32):
-            assert kq.kq_kernel_name(n1, n2, True) == "kq_warp_mma_kernel"
     assert kq.kq_kernel_for(4096, 64, 80, True, 0.85) == "kq_tc05_fused_kernel"     # hidden5120
-    assert kq.kq_kernel_for(64, 16, 16, False, 0.9) == "kq_warp_mma_kernel"         # tiny
+    assert kq.kq_kernel_for(64, 16, 16, False, 0.9) == "kq_tc05_fused_kernel"       # tiny
     assert kq.kq_kernel_for(64, 64, 64, False, 1e-7) == "kq_warp_mma_kernel"
 
 
