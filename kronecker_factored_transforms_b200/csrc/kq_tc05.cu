@@ -159,9 +159,16 @@ struct Cfg {
     static constexpr int N1P = align_up(N1, 32);     // TMEM columns of a D2 region
     static constexpr int R1W = align_up(NS1, 32);    // TMEM columns of a D1/A2 region
     // P2^T lives in TMEM (stage 1 reads A from TMEM) when the columns allow it.
-    static constexpr bool A1_TMEM = N1P <= 96;
+    // With cinv and n1 > 96 it does so at the cost of a single D2 region that the
+    // two epilogue warpgroups take in turn (SHARED_D2): stage 1's two passes then
+    // read only the x' tiles from shared memory, which bounds that case.
+    // (not at n1 = 128 with a padded n2, which runs short of registers that way)
+    static constexpr bool SHARED_D2 = SCALED && N1 > 96 && !(N1 == 128 && PADDED);
+    static constexpr bool A1_TMEM = N1P <= 96 || SHARED_D2;
     static constexpr int A1COLS = A1_TMEM ? 64 : 0;  // 128 K-elements of bf16
-    static constexpr int NB2 = (A1COLS + 2 * R1W + 3 * N1P <= 512) ? 3 : 2;       // D2 regions (groups)
+    static constexpr int NB2 = SHARED_D2 ? 1 : ((A1COLS + 2 * R1W + 3 * N1P <= 512) ? 3 : 2);  // D2 regions
+    // D2FULL barriers: one per D2 region, or with SHARED_D2 one per epilogue warpgroup
+    static constexpr int ND2F = SHARED_D2 ? 2 : NB2;
     static constexpr int NB1 = imin(4, (512 - A1COLS - NB2 * N1P) / R1W);        // D1/A2 regions (batches)
     static constexpr int TMEM_USED = A1COLS + NB1 * R1W + NB2 * N1P;
     static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
@@ -177,7 +184,7 @@ struct Cfg {
     static constexpr int SC = (SCALED && BUDGET >= 10 * XTILE) ? 4 : 2;  // lo-half tile stages (cinv)
     static constexpr int SX = imax(2, imin(8, (BUDGET - (SCALED ? SC * XTILE : 0)) / XTILE));  // raw x stages
     static constexpr int OFF_CONV = OFF_RAW + SX * XTILE;
-    static constexpr int NBAR = 2 * SX + 2 * SC + 3 * NB1 + 2 * NB2 + 2;
+    static constexpr int NBAR = 2 * SX + 2 * SC + 3 * NB1 + ND2F + NB2 + 2;
     // P1 and P2 arrive first, by bulk copies into the last NSCR x stages, which
     // take x tiles only once the factor operands are built from them.  With cinv
     // and n1 >= 112 only two x stages fit; the scratch then takes the lo-half
@@ -195,7 +202,7 @@ struct Cfg {
     // barrier indices
     static constexpr int FULL = 0, EMPTY = SX, CFULL = 2 * SX, CEMPTY = 2 * SX + SC;
     static constexpr int D1FULL = 2 * SX + 2 * SC, A2FULL = D1FULL + NB1, D1EMPTY = A2FULL + NB1;
-    static constexpr int D2FULL = D1EMPTY + NB1, D2EMPTY = D2FULL + NB2, TEARDOWN = D2EMPTY + NB2;
+    static constexpr int D2FULL = D1EMPTY + NB1, D2EMPTY = D2FULL + ND2F, TEARDOWN = D2EMPTY + NB2;
     static constexpr int FACT = TEARDOWN + 1;  // P1 and P2 landed in the scratch
     static_assert(SX > NSCR_RAW && NSCR - NSCR_RAW <= (SCALED ? SC : 0) , "at least one x stage besides the factor scratch");
     static_assert(N2 % 16 == 0 && N2 >= 16 && N2 <= 128, "stage 1 needs K = H * n2 (padded) = 128");
@@ -287,8 +294,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(bar(C::A2FULL + b), 128);
             mbar_init(bar(C::D1EMPTY + b), 1);
         }
+        for (int b = 0; b < C::ND2F; ++b) mbar_init(bar(C::D2FULL + b), 1);
         for (int b = 0; b < C::NB2; ++b) {
-            mbar_init(bar(C::D2FULL + b), 1);
             mbar_init(bar(C::D2EMPTY + b), 128);
         }
         mbar_init(bar(C::TEARDOWN), 2);  // one commit from each MMA issuer
@@ -541,6 +548,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
         } else {
             Ring r1p, r2;  // D1/A2 regions, D2 regions
+            uint32_t li = 0;  // groups issued (SHARED_D2: D2FULL of warpgroup li % 2)
             for (int64_t j = 0; j < nb; ++j) {
                 bool ok = wait_bounded(bar(C::A2FULL + r1p.idx), r1p.phase, s_abort, kSiteMma, kWaitLimitNs, false);
                 if (!__all_sync(0xffffffffu, ok)) break;
@@ -564,10 +572,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                     mma_ts_split<0>(d2, a2 + 16 * kk + 8 * pass, b2l + koff2(kk), kSdescSw128Hi,
                                                     idesc2);
                             }
-                        tc_commit(bar(C::D2FULL + r2.idx));
+                        tc_commit(bar(C::D2FULL + (C::SHARED_D2 ? (li & 1u) : r2.idx)));
                     }
                     __syncwarp();
                     r2.next(C::NB2);
+                    ++li;
                 }
                 if (!ok) break;
                 if (elect_one()) tc_commit(bar(C::D1EMPTY + r1p.idx));  // A2 region free
@@ -835,7 +844,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t jb = gi / C::GB, gp = gi % C::GB;
             const int64_t g = (int64_t(blockIdx.x) + int64_t(jb) * gridDim.x) * C::GB + gp;
             const int buf = it & 1;
-            const bool ok = wait_bounded(bar(C::D2FULL + b), ph, s_abort, kSiteEpilogue, kWaitLimitNs, false);
+            const bool ok = wait_bounded(bar(C::D2FULL + (C::SHARED_D2 ? uint32_t(ew) : b)),
+                                         C::SHARED_D2 ? uint32_t(it & 1) : ph, s_abort, kSiteEpilogue, kWaitLimitNs,
+                                         false);
             // All four warps leave together, so none is left behind in a named barrier.
             const bool warp_ok = __all_sync(0xffffffffu, ok);
             if (named_barrier_any(nbar, 128, !warp_ok)) break;
