@@ -65,7 +65,12 @@ typedef enum kq_status {
 typedef struct CUstream_st *kq_stream_t;
 
 /*
- * kq_transform_quant -- the fused hot path.
+ * kq_transform_quant -- the fused hot path.  Every supported shape runs on the
+ * tensor cores (alpha >= 2^-19): short launches at n1 = 64, n2 in {64, 128} in
+ * the pair-pipelined kernel, everything else in the batch-pipelined kernel
+ * (n2 = 16, 32, 48 padded to 64 columns per token, 80, 96, 112 to 128);
+ * kq_kernel_for names the kernel a call runs.  alpha below 2^-19 runs on the
+ * warp-level MMA kernel.
  *   x         [T, n1*n2] bf16, 16-byte aligned.
  *   P1        [n1, n1] bf16 (left factor; applied transposed), 16-byte aligned.
  *   P2        [n2, n2] bf16 (right factor), 16-byte aligned.
@@ -290,16 +295,19 @@ const char *kq_status_string(int status);
 
 /*
  * Name of the kernel kq_transform_quant launches for this shape on long inputs
- * (static storage), or "unsupported".  Host-only; touches no device state.
+ * (static storage): "kq_tc05_fused_kernel" for every supported shape, or
+ * "unsupported".  Host-only; touches no device state.
  */
 const char *kq_kernel_name(int n1, int n2, int has_cinv);
 
 /*
  * Name of the kernel kq_transform_quant launches for this call size (T tokens)
  * and clip ratio on the current device (static storage), or "unsupported".
- * Short launches of n1 = 64 (at most 24 groups of 128/n2 tokens per SM) run
- * kq_fused_kernel, the group-pipelined kernel; longer ones the kernel that
- * kq_kernel_name names.  Reads the device's SM count; launches nothing.
+ * Short launches of n1 = 64 and n2 in {64, 128} (at most 24 groups of 128/n2
+ * tokens per SM) run kq_fused_kernel, the pair-pipelined kernel; longer ones
+ * and every other shape the kernel that kq_kernel_name names; alpha below
+ * 2^-19 kq_warp_mma_kernel.  Reads the device's SM count (148 when no device
+ * is visible); launches nothing.
  */
 const char *kq_kernel_for(int64_t T, int n1, int n2, int has_cinv, float alpha);
 

@@ -74,9 +74,11 @@ kq_status device_info(DeviceInfo &info) {
 enum class Kern { Fused, Tc05, WarpMma };
 Kern choose_kernel(int64_t T, int n1, int n2, bool scaled, float alpha, bool quant, int num_sms) {
     if (!quant || !(alpha >= 0x1p-19f)) return Kern::WarpMma;  // fp32 y out, or the rounding's range
-    const int64_t groups = (T + (128 / (n2 >= 64 ? n2 : 64)) - 1) / (128 / (n2 >= 64 ? n2 : 64));
-    const bool rows_ok = T * int64_t(n1) < (int64_t(1) << 31);  // TMA row coordinates are 32-bit
-    if (rows_ok && kq::fused_supports(n1, n2, scaled) && groups <= int64_t(24) * num_sms) return Kern::Fused;
+    // tokens per group: 128 / (n2 padded to 64 or 128)
+    const int64_t h = n2 <= 64 ? 2 : 1, groups = (T + h - 1) / h;
+    // TMA row coordinates are 32-bit: past 2^31 rows of x both tensor-core kernels give way
+    if (T * int64_t(n1) >= (int64_t(1) << 31)) return Kern::WarpMma;
+    if (kq::fused_supports(n1, n2, scaled) && groups <= int64_t(24) * num_sms) return Kern::Fused;
     if (kq::tc05_supports(n1, n2, scaled)) return Kern::Tc05;
     return Kern::WarpMma;
 }

@@ -74,6 +74,9 @@ def test_kernel_selection_rules(kq):
     assert kq.kq_kernel_for(16, 112, 128, False, 0.9) == tc
     assert kq.kq_kernel_for(16, 64, 64, False, 2.0 ** -20) == warp  # alpha below 2^-19
     assert kq.kq_kernel_for(16, 24, 64, False, 0.9) == "unsupported"
+    # 2^31 rows of x or more: past the 32-bit TMA row coordinates, the warp-MMA kernel
+    assert kq.kq_kernel_for(2 ** 31 // 64 - 1, 64, 128, True, 0.85) == tc
+    assert kq.kq_kernel_for(2 ** 31 // 64, 64, 128, True, 0.85) == warp
 
 
 # Fake, never-dereferenced device addresses (validation rejects every call below).
