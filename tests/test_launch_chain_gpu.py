@@ -29,10 +29,14 @@ def dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-@pytest.mark.parametrize("name,T1,T2", [("hidden8192", 4096, 8192),   # tcgen05 kernel, 64 x 128, cinv
-                                         ("tiny", 16384, 32768)])       # warp-MMA kernel, 16 x 16
-def test_transform_chain_war_and_raw(kq, name, T1, T2):
+@pytest.mark.parametrize("name,T1,T2,alpha", [
+    ("hidden8192", 4096, 8192, None),         # batch, batch, then pair kernel (T3 = 2048): 64 x 128, cinv
+    ("hidden8192", 2048, 8192, None),         # pair, batch, pair
+    ("tiny", 16384, 32768, None),             # batch kernel with n2 = 16 padded to 64 columns
+    ("llama7b_hidden", 1024, 4096, 2.0 ** -20)])  # warp-MMA kernel (alpha below 2^-19)
+def test_transform_chain_war_and_raw(kq, name, T1, T2, alpha):
     w = make_workload(name, T=T1)
+    alpha = w.alpha if alpha is None else alpha
     n1, n2, n = w.n1, w.n2, w.n
     xA0 = dev(w.x.view(np.int16))
     xB = dev(make_workload(name, T=T2, shard=1).x.view(np.int16))
@@ -46,13 +50,17 @@ def test_transform_chain_war_and_raw(kq, name, T1, T2):
     q2 = xA.view(torch.uint8)[: T2 * n // 2]          # call 2 writes its codes over call 1's input
 
     def call1():
-        kq.kq_transform_quant(xA, P1, P2, cinv, w.alpha, q1, s1, T1, n1, n2)
+        kq.kq_transform_quant(xA, P1, P2, cinv, alpha, q1, s1, T1, n1, n2)
 
     def call2():
-        kq.kq_transform_quant(xB, P1, P2, cinv, w.alpha, q2, s2, T2, n1, n2)
+        kq.kq_transform_quant(xB, P1, P2, cinv, alpha, q2, s2, T2, n1, n2)
 
     def call3():
-        kq.kq_transform_quant(q2, P1, P2, None, w.alpha, q3, s3, T3, n1, n2)
+        kq.kq_transform_quant(q2, P1, P2, None, alpha, q3, s3, T3, n1, n2)
+
+    kinds = [kq.kq_kernel_for(t, n1, n2, c, alpha) for t, c in ((T1, cinv is not None), (T2, cinv is not None),
+                                                                (T3, False))]
+    assert "unsupported" not in kinds
 
     def snap():
         return [t.clone() for t in (q1, s1, q2, s2, q3, s3)]
