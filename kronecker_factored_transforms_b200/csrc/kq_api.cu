@@ -65,7 +65,7 @@ kq_status device_info(DeviceInfo &info) {
     return KQ_OK;
 }
 
-// Which transform kernel a quantising call of this size runs.  The group-pipelined
+// Which transform kernel a quantising call of this size runs.  The pair-pipelined
 // kernel (n1 = 64) wins on short launches -- up to about 24 groups of 128 / n2
 // tokens per SM, where its short start-up and per-group pipeline matter most -- and
 // the batch-pipelined tcgen05 kernel on long ones (measured on B200: 4.1 against

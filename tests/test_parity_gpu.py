@@ -247,7 +247,7 @@ def test_dequant_inverse_matches_oracle_and_round_trips(kq):
 # Kernel selection and the bounded-wait failure path.
 
 def test_fast_kernel_is_selected_for_the_configs(kq):
-    # long launches: the batch-pipelined kernel; short ones of n1 = 64: the group-pipelined one
+    # long launches: the batch-pipelined kernel; short ones of n1 = 64: the pair-pipelined one
     for n1, n2, scaled in [(64, 64, False), (64, 128, True), (112, 128, False)]:
         assert kq.kq_kernel_name(n1, n2, scaled) == "kq_tc05_fused_kernel"
     assert kq.kq_kernel_for(8192, 64, 128, True, 0.85) == "kq_tc05_fused_kernel"   # hidden8192
