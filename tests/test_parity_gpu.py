@@ -149,6 +149,19 @@ def test_shapes_ragged(kq, n1, n2, scaled):
     assert_quant_parity(x, P1, P2, cinv, alpha, n1, n2, q, s)
 
 
+@pytest.mark.parametrize("name,T", [("hidden8192", 148 * 24), ("hidden8192", 148 * 24 + 1),
+                                    ("llama7b_hidden", 148 * 48), ("llama7b_hidden", 148 * 48 + 2)])
+def test_dispatch_boundary(kq, name, T):
+    """The last size of the pair-pipelined kernel (24 groups per SM on 148 SMs) and
+    the first of the batch-pipelined one, both against the oracle."""
+    w = make_workload(name, T=T)
+    expect = "kq_fused_kernel" if (T + 128 // w.n2 - 1) // (128 // w.n2) <= 24 * 148 else "kq_tc05_fused_kernel"
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert kq.kq_kernel_for(T, w.n1, w.n2, w.cinv is not None, w.alpha) == expect
+    q, s = run_quant(kq, w.x, w.P1, w.P2, w.cinv, w.alpha, T, w.n1, w.n2)
+    assert_quant_parity(w.x, w.P1, w.P2, w.cinv, w.alpha, w.n1, w.n2, q, s)
+
+
 @pytest.mark.parametrize("T", [1, 2, 3, 7])
 def test_small_T(kq, T):
     w = make_workload("hidden8192", rows=T)
