@@ -66,8 +66,9 @@ typedef struct CUstream_st *kq_stream_t;
 
 /*
  * kq_transform_quant -- the fused hot path.  Every supported shape runs on the
- * tensor cores (alpha >= 2^-19): short launches at n1 = 64, n2 in {64, 128} in
- * the pair-pipelined kernel, everything else in the batch-pipelined kernel
+ * tensor cores (alpha >= 2^-19): short launches at n1 = 64, n2 in {64, 128}
+ * (up to 56 groups of 128/n2 tokens per SM without cinv, 4 with it) in the
+ * pair-pipelined kernel, everything else in the batch-pipelined kernel
  * (n2 = 16, 32, 48 padded to 64 columns per token, 80, 96, 112 to 128);
  * kq_kernel_for names the kernel a call runs.  alpha below 2^-19 runs on the
  * warp-level MMA kernel.
@@ -303,8 +304,9 @@ const char *kq_kernel_name(int n1, int n2, int has_cinv);
 /*
  * Name of the kernel kq_transform_quant launches for this call size (T tokens)
  * and clip ratio on the current device (static storage), or "unsupported".
- * Short launches of n1 = 64 and n2 in {64, 128} (at most 24 groups of 128/n2
- * tokens per SM) run kq_fused_kernel, the pair-pipelined kernel; longer ones
+ * Short launches of n1 = 64 and n2 in {64, 128} (at most 56 groups of 128/n2
+ * tokens per SM without cinv, 4 with it) run kq_fused_kernel, the pair-pipelined
+ * kernel; longer ones
  * and every other shape the kernel that kq_kernel_name names; alpha below
  * 2^-19 kq_warp_mma_kernel.  Reads the device's SM count (148 when no device
  * is visible); launches nothing.

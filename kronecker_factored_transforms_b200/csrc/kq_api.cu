@@ -66,11 +66,12 @@ kq_status device_info(DeviceInfo &info) {
 }
 
 // Which transform kernel a quantising call of this size runs.  The pair-pipelined
-// kernel (n1 = 64) wins on short launches -- up to about 24 groups of 128 / n2
-// tokens per SM, where its short start-up and per-group pipeline matter most -- and
-// the batch-pipelined tcgen05 kernel on long ones (measured on B200: 4.1 against
-// 5.0 us at T = 1, 9.0 against 9.4 us at 2048 x 64x64, 47 against 56 us at
-// 8192 x 64x128 with cinv).
+// kernel (n1 = 64) wins on short launches, where its short start-up and per-group
+// pipeline matter most, and the batch-pipelined tcgen05 kernel on long ones.  The
+// crossover, measured on B200: without cinv about 56 groups of 128 / n2 tokens per
+// SM (64x64: 25.2 against 25.8 us at T = 10000, 39.4 against 39.9 at 16384, 152
+// against 148 at 65536); with cinv about 4 (64x128: 6.6 against 6.7 us at T = 256,
+// 8.0 both at 512, 11.8 against 11.1 at 1024, 19.5 against 15.3 at 2048).
 enum class Kern { Fused, Tc05, WarpMma };
 Kern choose_kernel(int64_t T, int n1, int n2, bool scaled, float alpha, bool quant, int num_sms) {
     if (!quant || !(alpha >= 0x1p-19f)) return Kern::WarpMma;  // fp32 y out, or the rounding's range
@@ -78,7 +79,8 @@ Kern choose_kernel(int64_t T, int n1, int n2, bool scaled, float alpha, bool qua
     const int64_t h = n2 <= 64 ? 2 : 1, groups = (T + h - 1) / h;
     // TMA row coordinates are 32-bit: past 2^31 rows of x both tensor-core kernels give way
     if (T * int64_t(n1) >= (int64_t(1) << 31)) return Kern::WarpMma;
-    if (kq::fused_supports(n1, n2, scaled) && groups <= int64_t(24) * num_sms) return Kern::Fused;
+    const int64_t per_sm = scaled ? 4 : 56;
+    if (kq::fused_supports(n1, n2, scaled) && groups <= per_sm * num_sms) return Kern::Fused;
     if (kq::tc05_supports(n1, n2, scaled)) return Kern::Tc05;
     return Kern::WarpMma;
 }

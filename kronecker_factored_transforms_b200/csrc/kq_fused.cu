@@ -1,8 +1,8 @@
 // kq_fused.cu -- persistent fused Kronecker transform + INT4 kernel on the
 // 5th-generation tensor cores, pipelined per pair of token groups; the kernel
-// kq_transform_quant runs for short launches at n1 = 64 (at most 24 groups
-// per SM), where the batch-pipelined kernel of kq_tc05.cu spends a larger
-// share of the launch filling and draining its pipeline.
+// kq_transform_quant runs for short launches at n1 = 64 (up to 56 groups per
+// SM without cinv, 4 with it), where the batch-pipelined kernel of kq_tc05.cu
+// spends a larger share of the launch filling and draining its pipeline.
 //
 // Method (FlatQuant page, "Kronecker factorization", "Per-channel scaling and
 // learnable clipping" and "The fused kernel"): per token Y~ = P1^T X~ P2 with

@@ -66,10 +66,12 @@ def test_kernel_selection_rules(kq):
         assert kq.kq_kernel_name(112, n2, True) == tc
         assert kq.kq_kernel_name(16, n2, False) == tc
     assert kq.kq_kernel_for(2048, 64, 64, False, 0.88) == pair      # short launch at n1 = 64
-    assert kq.kq_kernel_for(148 * 24, 64, 128, True, 0.85) == pair  # 24 groups per SM
-    assert kq.kq_kernel_for(148 * 24 + 1, 64, 128, True, 0.85) == tc
-    assert kq.kq_kernel_for(148 * 48, 64, 64, False, 0.9) == pair   # two tokens per group at n2 = 64
-    assert kq.kq_kernel_for(148 * 48 + 2, 64, 64, False, 0.9) == tc
+    assert kq.kq_kernel_for(148 * 4, 64, 128, True, 0.85) == pair   # with cinv: 4 groups per SM
+    assert kq.kq_kernel_for(148 * 4 + 1, 64, 128, True, 0.85) == tc
+    assert kq.kq_kernel_for(148 * 56, 64, 128, False, 0.9) == pair  # without: 56 groups per SM
+    assert kq.kq_kernel_for(148 * 56 + 1, 64, 128, False, 0.9) == tc
+    assert kq.kq_kernel_for(148 * 112, 64, 64, False, 0.9) == pair  # two tokens per group at n2 = 64
+    assert kq.kq_kernel_for(148 * 112 + 2, 64, 64, False, 0.9) == tc
     assert kq.kq_kernel_for(16, 64, 80, True, 0.85) == tc           # the pair kernel has n2 in {64, 128} only
     assert kq.kq_kernel_for(16, 112, 128, False, 0.9) == tc
     assert kq.kq_kernel_for(16, 64, 64, False, 2.0 ** -20) == warp  # alpha below 2^-19

@@ -149,13 +149,15 @@ def test_shapes_ragged(kq, n1, n2, scaled):
     assert_quant_parity(x, P1, P2, cinv, alpha, n1, n2, q, s)
 
 
-@pytest.mark.parametrize("name,T", [("hidden8192", 148 * 24), ("hidden8192", 148 * 24 + 1),
-                                    ("llama7b_hidden", 148 * 48), ("llama7b_hidden", 148 * 48 + 2)])
+@pytest.mark.parametrize("name,T", [("hidden8192", 148 * 4), ("hidden8192", 148 * 4 + 1),
+                                    ("llama7b_hidden", 148 * 112), ("llama7b_hidden", 148 * 112 + 2)])
 def test_dispatch_boundary(kq, name, T):
-    """The last size of the pair-pipelined kernel (24 groups per SM on 148 SMs) and
-    the first of the batch-pipelined one, both against the oracle."""
+    """The last size of the pair-pipelined kernel (on 148 SMs: 4 groups per SM with
+    cinv, 56 without) and the first of the batch-pipelined one, both against the oracle."""
     w = make_workload(name, T=T)
-    expect = "kq_fused_kernel" if (T + 128 // w.n2 - 1) // (128 // w.n2) <= 24 * 148 else "kq_tc05_fused_kernel"
+    per_sm = 4 if w.cinv is not None else 56
+    expect = ("kq_fused_kernel" if (T + 128 // w.n2 - 1) // (128 // w.n2) <= per_sm * 148
+              else "kq_tc05_fused_kernel")
     if torch.cuda.get_device_properties(0).multi_processor_count == 148:
         assert kq.kq_kernel_for(T, w.n1, w.n2, w.cinv is not None, w.alpha) == expect
     q, s = run_quant(kq, w.x, w.P1, w.P2, w.cinv, w.alpha, T, w.n1, w.n2)
@@ -266,6 +268,7 @@ def test_fast_kernel_is_selected_for_the_configs(kq):
     assert kq.kq_kernel_for(8192, 64, 128, True, 0.85) == "kq_tc05_fused_kernel"   # hidden8192
     assert kq.kq_kernel_for(65536, 64, 64, False, 0.9) == "kq_tc05_fused_kernel"   # sweep4096, largest T
     assert kq.kq_kernel_for(2048, 64, 64, False, 0.88) == "kq_fused_kernel"        # llama7b_hidden
+    assert kq.kq_kernel_for(2048, 64, 128, True, 0.85) == "kq_tc05_fused_kernel"   # with cinv: 14 groups per SM
     assert kq.kq_kernel_for(1, 64, 128, True, 0.85) == "kq_fused_kernel"
     assert kq.kq_kernel_for(4096, 112, 128, False, 0.9) == "kq_tc05_fused_kernel"  # mlp14336
     for n1 in (16, 48, 64, 80, 96, 112, 128):  # cinv with n1 > 64; n2 padded to 64 or 128
