@@ -22,8 +22,12 @@
 // (|sum| <= 16384 K < 2^31); the epilogue shifts the factor out and applies
 // (float(sum) * sx[m]) * sw[o].
 //
-// One CTA per 128 x 256 output tile.  Warps: 0 TMA producer | 1 TMEM
-// allocator + MMA issuer | 4-11 expanders, then the epilogue | 2-3 idle.
+// One CTA per 256 x 128 output tile: two 128-row activation tiles in TMEM (the
+// A operands of two MMAs) share one widened weight tile in shared memory, so
+// each widened weight byte written to shared memory feeds two MMAs; that keeps
+// the shared-memory traffic per output a seventh below a 128 x 256 tile's.
+// Warps: 0 TMA producer | 1 TMEM allocator + MMA issuer | 4-11 expanders, then
+// the epilogue | 2-3 idle.
 // Every mbarrier wait is bounded (kq_wait.cuh).
 #include <mutex>
 
@@ -37,21 +41,21 @@ namespace {
 
 using namespace tc;
 
-constexpr int TM = 128, TN = 256, KC = 128;            // tile rows, columns, codes per K chunk
-constexpr int PA = TM * KC / 2, PB = TN * KC / 2;       // packed bytes per chunk: 8 KB, 16 KB
-constexpr int EB = TN * KC;                             // widened int8 weight bytes per chunk: 32 KB
-constexpr int NS = 4, NE = 3;                           // packed stages, widened stages
+constexpr int TM = 256, TN = 128, KC = 128;            // tile rows (two MMA tiles), columns, codes per K chunk
+constexpr int PA = TM * KC / 2, PB = TN * KC / 2;       // packed bytes per chunk: 16 KB, 8 KB
+constexpr int EB = TN * KC;                             // widened int8 weight bytes per chunk: 16 KB
+constexpr int NS = 5, NE = 4;                           // packed stages, widened stages
 constexpr int G_THREADS = 384;                          // 12 warps
 constexpr int XW0 = 4, NXW = 8;                         // expander / epilogue warps 4-11
-constexpr int OFF_E = NS * (PA + PB);                   // 96 KB: widened weight stages (1024-aligned)
+constexpr int OFF_E = NS * (PA + PB);                   // 120 KB: widened weight stages (1024-aligned)
 constexpr int OFF_BAR = OFF_E + NE * EB;
 constexpr int FULL = 0, EMPTY = NS, XFULL = 2 * NS, XEMPTY = 2 * NS + NE, DONE = 2 * NS + 2 * NE;
 constexpr int NBAR = DONE + 1;
 constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;            // TMEM base, abort flag
 constexpr int G_SMEM = OFF_MISC + 16 + 1024;            // + slack for 1024-byte alignment
-constexpr uint32_t TMEM_COLS = 512;                     // s32 accumulator [0, 256) + widened activations
-constexpr uint32_t ACOL = TN;                           // widened activation stage e at columns 256 + 32 e
-static_assert(ACOL + NE * (KC / 4) <= TMEM_COLS, "TMEM budget");
+constexpr uint32_t TMEM_COLS = 512;  // s32 accumulators [0, 128) and [128, 256) + widened activations
+constexpr uint32_t ACOL = 2 * TN;    // widened activation stage e: tile h at columns 256 + 64 e + 32 h
+static_assert(ACOL + NE * 2 * (KC / 4) <= TMEM_COLS, "TMEM budget");
 static_assert(OFF_E % 1024 == 0 && EB % 1024 == 0 && (PA + PB) % 1024 == 0, "swizzle atoms");
 static_assert(G_SMEM <= 227 * 1024, "shared memory budget");
 
@@ -176,7 +180,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
-        constexpr uint32_t idesc = idesc_s8_s32(TM, TN);
+        constexpr uint32_t idesc = idesc_s8_s32(128, TN);
         Ring r;
         for (int kt = 0; kt < KT; ++kt, r.next(NE)) {
             const bool ok = wait_bounded_err(bar(XFULL + r.idx), r.phase, s_abort, kSiteGemm, kWaitLimitNs, false,
@@ -184,14 +188,18 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const uint32_t bl = sdesc_sw128_lo(sbase + uint32_t(OFF_E + r.idx * EB));
-            const uint32_t at = tmem + ACOL + uint32_t(r.idx * (KC / 4));
+            const uint32_t at = tmem + ACOL + uint32_t(r.idx * 2 * (KC / 4));
             if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < KC / 32; ++kk) {  // K = 32 int8 per MMA: 8 TMEM columns, +32 bytes of B
-                    if ((kt | kk) != 0)
-                        mma_i8_ts<1>(tmem, at + 8 * kk, bl + 2 * kk, idesc);
-                    else
-                        mma_i8_ts<0>(tmem, at + 8 * kk, bl + 2 * kk, idesc);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {      // the two 128-row tiles share the B slice
+                        const uint32_t d = tmem + uint32_t(h * TN), a = at + uint32_t(h * (KC / 4)) + 8 * kk;
+                        if ((kt | kk) != 0)
+                            mma_i8_ts<1>(d, a, bl + 2 * kk, idesc);
+                        else
+                            mma_i8_ts<0>(d, a, bl + 2 * kk, idesc);
+                    }
                 }
                 tc_commit(bar(XEMPTY + r.idx));  // widened stage free once these MMAs complete
             }
@@ -204,17 +212,17 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         __syncwarp();
     } else if (warp >= XW0 && warp < XW0 + NXW) {
         // ---------------- expanders: packed INT4 -> int8 (x16) ----------------
-        // Activations: thread (warp w, lane) widens half (hh = (w - 4) / 4) of
-        // row m = 32 (w % 4) + lane: two 16-byte units of the packed tile (64B
-        // swizzle: unit c of row m at m * 64 + 16 (c ^ ((m >> 1) & 3)), so the
-        // eight rows of a shared-memory phase hit eight bank groups) become
-        // sixteen TMEM columns of lane m.  Weights: four 16-byte units per thread
-        // into the 128B-swizzled K-major shared tile.
+        // Activations: thread (warp w, lane) widens row am = 128 hh + 32 (w % 4) +
+        // lane of the 256-row tile (hh = (w - 4) / 4): its four 16-byte units of
+        // the packed tile (64B swizzle: unit c of row m at m * 64 + 16 (c ^ ((m >> 1)
+        // & 3)), so the eight rows of a shared-memory phase hit eight bank groups)
+        // become 32 TMEM columns of lane am % 128 in MMA tile hh.  Weights: two
+        // 16-byte units per thread into the 128B-swizzled K-major shared tile.
         const int xt = tid - XW0 * 32;                // 0 .. 255
         const int hh = (warp - XW0) >> 2, qa = warp & 3;
-        const int am = 32 * qa + lane;                // activation row = TMEM lane
-        constexpr int UB = TN * (KC / 32);            // 16-byte packed weight units per chunk: 1024
-        constexpr int UPB = UB / (NXW * 32);          // 4 per thread
+        const int am = 128 * hh + 32 * qa + lane;     // activation row of the tile
+        constexpr int UB = TN * (KC / 32);            // 16-byte packed weight units per chunk: 512
+        constexpr int UPB = UB / (NXW * 32);          // 2 per thread
         static_assert(UB % (NXW * 32) == 0, "unit split");
         Ring rs, re;
         bool ok = true;
@@ -226,27 +234,27 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             tc_fence_after();
             const unsigned char *pk = smem + rs.idx * (PA + PB);
             unsigned char *ex = smem + OFF_E + re.idx * EB;
-            uint4 va[2], vb[UPB];
+            uint4 va[4], vb[UPB];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const int u = 2 * hh + c;
-                va[c] = *reinterpret_cast<const uint4 *>(pk + am * 64 + ((u ^ ((am >> 1) & 3)) << 4));
-            }
+            for (int c = 0; c < 4; ++c)
+                va[c] = *reinterpret_cast<const uint4 *>(pk + am * 64 + ((c ^ ((am >> 1) & 3)) << 4));
 #pragma unroll
             for (int i = 0; i < UPB; ++i)
                 vb[i] = *reinterpret_cast<const uint4 *>(pk + PA + (xt + i * NXW * 32) * 16);
-            // activations -> TMEM: unit c gives columns 8 c .. 8 c + 7 of this half
-            uint32_t o[16];
+            // activations -> TMEM: unit c gives columns 8 c .. 8 c + 7 of this row's tile
+            uint32_t o[2][16];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 const uint32_t w[4] = {va[c].x, va[c].y, va[c].z, va[c].w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    o[8 * c + 2 * j] = (w[j] << 4) & 0xF0F0F0F0u;  // even codes of the 8-code group, x16
-                    o[8 * c + 2 * j + 1] = w[j] & 0xF0F0F0F0u;     // odd codes, x16
+                    o[c >> 1][8 * (c & 1) + 2 * j] = (w[j] << 4) & 0xF0F0F0F0u;  // even codes of the 8-code group, x16
+                    o[c >> 1][8 * (c & 1) + 2 * j + 1] = w[j] & 0xF0F0F0F0u;     // odd codes, x16
                 }
             }
-            tmem_st_32x32b_x16(tmem + (uint32_t(32 * qa) << 16) + ACOL + uint32_t(re.idx * (KC / 4) + 16 * hh), o);
+            const uint32_t tcol = tmem + (uint32_t(32 * qa) << 16) + ACOL + uint32_t((2 * re.idx + hh) * (KC / 4));
+            tmem_st_32x32b_x16(tcol, o[0]);
+            tmem_st_32x32b_x16(tcol + 16, o[1]);
             // weights -> shared memory
 #pragma unroll
             for (int i = 0; i < UPB; ++i) {
@@ -275,19 +283,19 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         const bool done = wait_bounded_err(bar(DONE), 0u, s_abort, kSiteGemm, kWaitLimitNs, false, err);
         if (__all_sync(0xffffffffu, done && ok)) {
             tc_fence_after();
-            const int q = warp & 3, h = (warp - XW0) >> 2;  // lane quarter, column half
-            const int64_t m = m0 + 32 * q + lane;
+            const int q = warp & 3, h = (warp - XW0) >> 2;  // lane quarter, 128-row tile
+            const int64_t m = m0 + 128 * h + 32 * q + lane;
             const float fx = m < M ? sx[m] : 0.0f;
             constexpr int OB = BF16 ? 2 : 4;  // output bytes per element
             void *yrow = static_cast<unsigned char *>(y) + (m < M ? m : 0) * N * OB;
             // vector stores only where every row start is aligned for them
             const bool vec = (N % 4) == 0 && (reinterpret_cast<uintptr_t>(y) & (4 * OB - 1)) == 0;
 #pragma unroll 1
-            for (int c = 0; c < TN / 2 / 32; ++c) {
+            for (int c = 0; c < TN / 32; ++c) {
                 uint32_t a[32];
-                tmem_ld_32x32b_x32(tmem + (uint32_t(32 * q) << 16) + uint32_t(128 * h + 32 * c), a);
+                tmem_ld_32x32b_x32(tmem + (uint32_t(32 * q) << 16) + uint32_t(TN * h + 32 * c), a);
                 tmem_wait_ld();
-                const int64_t nb = n0 + 128 * h + 32 * c;
+                const int64_t nb = n0 + 32 * c;
                 if (m < M) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 4) {
