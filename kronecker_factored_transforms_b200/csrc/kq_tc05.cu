@@ -1,17 +1,19 @@
 // kq_tc05.cu -- persistent fused Kronecker transform + INT4 kernel on the
 // 5th-generation tensor cores (tcgen05.mma, accumulators in TMEM), pipelined
 // per batch of token groups: the kernel kq_transform_quant runs for long
-// launches and for n1 != 64 (kq_fused.cu takes short launches at n1 = 64);
-// plus the device status word that the bounded waits report through.
+// launches and for every shape but n1 = 64 with n2 in {64, 128} (kq_fused.cu
+// takes the short launches of those); plus the device status word that the
+// bounded waits report through.
 //
 // Method (FlatQuant page, "Kronecker factorization" and "The fused kernel"):
 // per token Y~ = P1^T X~ P2 with X~ the row-major n1 x n2 view of x * cinv,
 // then per-token absmax, s = alpha * max / 7, round-half-even codes clamped
 // to [-8, 7], packed two per byte.  Only codes and scales reach HBM.
 //
-// Layout of the work (one CTA per SM, 24 warps, groups of H = 128 / n2
-// tokens so that the 128 TMEM lanes always hold 128 output columns; stage 1
-// runs on batches of GB groups, MMAs up to 128 columns wide):
+// Layout of the work (one CTA per SM, 24 warps, groups of H = 128 / n2 tokens
+// so that the 128 TMEM lanes always hold 128 output columns -- n2 = 16, 32, 48
+// padded to 64 and 80, 96, 112 to 128, the padding zero; stage 1 runs on
+// batches of GB groups, MMAs up to 128 columns wide):
 //   TMEM lane l = (h, m): token h of the group, output column
 //   j = lane_column(m) of its n2 columns.  Within each block of 32 lanes the
 //   columns are interleaved so that the thread of a 16x256b TMEM load that
@@ -19,7 +21,8 @@
 //   columns, i.e. two whole output bytes.
 //   stage 1           D1[l][a]  = sum_(h',b) A1[l][(h',b)] * X[a][(h',b)]
 //                     A1 = block-diag over h of P2^T (rows permuted as above),
-//                     resident in TMEM (or shared memory for n1 > 96);
+//                     resident in TMEM (in shared memory for n1 > 96
+//                     without cinv, and at n1 = 128 with a padded n2);
 //                     X  = the group's x tile straight from TMA (K = 128).
 //   convert (TMEM)    D1 fp32 -> A2 = hi and -lo bf16, in place, chunk by chunk
 //                     (hi = the top 16 bits, -lo = hi - D1 by one mixed
@@ -27,12 +30,14 @@
 //   stage 2 (TS MMA)  D2[l][i]  = sum_a A2[l][a] * P1[a][i]   (A from TMEM; the
 //                     -lo pass with the MMA's negate-B bit)
 //   epilogue          absmax over the token's lanes, quantise, pack into a
-//                     swizzled staging tile, one TMA store per group to HBM.
+//                     swizzled staging tile, one TMA store per group to HBM
+//                     (padded n2: plain rows, one bulk copy per group).
 // With cinv, the x' split warps turn each raw x tile into x' = x * cinv
 // split into a hi bf16 tile (written over x) and a lo bf16 tile; stage 1
 // then accumulates both (for n1 > 64 the lo tile holds -lo and its pass
-// negates B).  TMEM holds P2^T, two D1/A2 regions (batches) and two or
-// three D2 regions (groups).
+// negates B).  TMEM holds P2^T, two D1/A2 regions (batches) and one to
+// three D2 regions (groups; one, taken in turn by the two epilogue
+// warpgroups, with cinv at n1 > 96).
 //
 // Warp roles: 0 TMA producer | 1 TMEM allocator + stage-1 MMA issuer | 5
 // stage-2 MMA issuer | 2-4, 6-7, 20, 22-23 x' split (cinv only) | 8-11 P2^T
