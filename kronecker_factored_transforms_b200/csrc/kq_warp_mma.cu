@@ -1,8 +1,9 @@
 // kq_warp_mma.cu -- general fused Kronecker transform + INT4 kernel on the
 // warp-level tensor-core path (mma.sync m16n8k16, bf16 in, fp32 accumulate).
 //
-// It covers every supported shape (n1, n2 multiples of 16 up to 128) and is
-// the reference GPU implementation the tcgen05 kernel is checked against.
+// It covers every supported shape (n1, n2 multiples of 16 up to 128) and runs
+// what the tcgen05 kernels do not: the fp32 check entry kq_transform, clip
+// ratios below 2^-19, and inputs of 2^31 rows of x or more.
 //
 // Method (FlatQuant page, "Kronecker factorization" and "The fused kernel"):
 // for a token, Y~ = P1^T X~ P2 with X~ the row-major n1 x n2 view of x * cinv.
