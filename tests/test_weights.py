@@ -11,8 +11,7 @@ import numpy as np
 import pytest
 
 from kronecker_factored_transforms_b200 import weights as kw
-from kronecker_factored_transforms_b200.workloads import (bf16_bits_to_f32, f32_to_bf16_bits, make_weights,
-                                                          make_workload)
+from kronecker_factored_transforms_b200.workloads import bf16_bits_to_f32, f32_to_bf16_bits, make_weights
 
 
 def test_svd_inverse_is_an_inverse():
